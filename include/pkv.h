@@ -1,0 +1,164 @@
+/*
+ * pkv.h - C ABI of libpkv.so: paged-KV decode attention for NVIDIA B200 (sm_100a).
+ *
+ * The problem these calls solve is the one stated on three pages about KV-cache
+ * memory management:
+ *   [mlqm]   "LLM推理显存优化KV Cache管理3大策略实测节省60%显存开销" (mlqm.cn/news/267625)
+ *   [gpuyard]"生产级 LLM 推理的 KV 缓存优化" (GPUYard repost on feinterview.poetries.top)
+ *   [yunthe] "大模型推理加速实战：KV Cache内存优化与PagedAttention分页管理方案" (yunthe.com)
+ *
+ * Memory layout (all device buffers, row-major, densely packed):
+ *   cache  k_cache, v_cache : [num_blocks][block_size][num_kv_heads][head_dim]
+ *          One physical block holds block_size token rows of all KV heads
+ *          ([mlqm] §2, the Block class: k_data/v_data of block_size x hidden).
+ *   scales k_scale, v_scale : fp32 [num_blocks][num_kv_heads][block_size]
+ *          (INT8 caches only; one scale per token per head, [mlqm] §4).
+ *   slot   physical_block * block_size + offset_in_block.
+ *   table  block_tables     : int32 [num_seqs][max_blocks_per_seq]; entry j is
+ *          the physical block of logical block j ([yunthe], PagedAttention
+ *          section, the block_table example; [mlqm] §2 BlockTable).
+ *
+ * Conventions shared by every call:
+ *   - The caller allocates and owns every buffer; the library keeps no state
+ *     between calls, allocates nothing and never synchronises.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and targets the current CUDA device.
+ *   - Argument errors return a negative pkv_status before anything is launched.
+ *   - Data errors found on the device (bad block id, bad slot, context length
+ *     out of range) are OR-ed as PKV_FLAG_* bits into *err_flag (a device int,
+ *     may be NULL); the offending token/row is skipped, the kernel never traps.
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pkv_stream_t; /* identical to cudaStream_t */
+
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_I8 = 2 } pkv_dtype;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_ARG = -1,         /* null pointer, negative size, n_q % n_kv != 0 */
+  PKV_ERR_DTYPE = -2,       /* unsupported dtype combination */
+  PKV_ERR_SHAPE = -3,       /* head_dim / block_size / group outside the supported set */
+  PKV_ERR_UNSUPPORTED = -4, /* no kernel for this configuration */
+  PKV_ERR_WORKSPACE = -5,   /* split-K needs a workspace of pkv_workspace_size() bytes */
+  PKV_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
+  PKV_ERR_ALIGN = -7        /* a device pointer is not 16-byte aligned */
+} pkv_status;
+
+/* Bits written into *err_flag by the kernels. */
+#define PKV_FLAG_BAD_BLOCK 1   /* block table entry outside [0, num_blocks): block skipped */
+#define PKV_FLAG_BAD_SLOT 2    /* slot >= num_blocks * block_size: token not written */
+#define PKV_FLAG_CTX_RANGE 4   /* context_len > max_blocks_per_seq * block_size or
+                                  > max_context_len: clamped */
+#define PKV_FLAG_NEG_CTX 8     /* negative context_len: treated as 0 */
+
+/* Supported sets: head_dim in {64, 128}; block_size a power of two in [8, 256];
+ * group = num_q_heads / num_kv_heads in [1, 16]. */
+
+/*
+ * pkv_kv_cache_append - write each new token's K and V into its cache slot.
+ *
+ * Defined by [yunthe] (KV-cache overhead section: every generated token's
+ * key/value is written into the KV cache) and [mlqm] §2 (block rows).  Token t
+ * with slot s = slot_mapping[t] goes to block s / block_size, row
+ * s % block_size; s < 0 skips the token (padding).  With cache_dt == PKV_I8 each
+ * (token, head) row of head_dim values is quantised as in [mlqm] §4
+ * (quantize_tensor): scale = 127 / max|x| over head_dim and code =
+ * clamp(rint(x * scale), -128, 127), all in fp32, round-half-to-even, no fused
+ * multiply-add; an all-zero row stores codes 0 and scale 1.  The scale goes to
+ * k_scale/v_scale[block][head][row].
+ *
+ *   k, v          device, [num_tokens][num_kv_heads][head_dim], dtype in_dt
+ *                 (PKV_F32 or PKV_BF16), contiguous.  Read only.
+ *   slot_mapping  device int64 [num_tokens].
+ *   k_cache, v_cache  device, cache layout above, dtype cache_dt (== in_dt, or PKV_I8).
+ *   k_scale, v_scale  device fp32 scale arrays; required iff cache_dt == PKV_I8.
+ *   err_flag      device int or NULL (PKV_FLAG_BAD_SLOT).
+ * Two tokens with the same slot race (last writer wins, unspecified).
+ */
+int pkv_kv_cache_append(const void* k, const void* v, const int64_t* slot_mapping,
+                        int num_tokens, int num_kv_heads, int head_dim, pkv_dtype in_dt,
+                        void* k_cache, void* v_cache, pkv_dtype cache_dt, int num_blocks,
+                        int block_size, float* k_scale, float* v_scale, int* err_flag,
+                        pkv_stream_t stream);
+
+/*
+ * pkv_decode_num_splits - the number of context splits (split-K partitions)
+ * pkv_paged_attention_decode picks when given num_splits = 0, for the current
+ * device.  Always >= 1.  Returns a negative pkv_status on bad arguments.
+ */
+int pkv_decode_num_splits(int num_seqs, int num_kv_heads, int head_dim, int max_context_len,
+                          pkv_dtype cache_dt);
+
+/*
+ * pkv_workspace_size - bytes of device workspace pkv_paged_attention_decode
+ * needs for this shape with `num_splits` splits (0 = the automatic choice).
+ * 0 when one split suffices (no workspace needed).
+ */
+size_t pkv_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                          int max_context_len, pkv_dtype cache_dt, int num_splits);
+
+/*
+ * pkv_paged_attention_decode - one decode step of attention over a paged cache.
+ *
+ * Defined by [yunthe], PagedAttention section: look up each token's physical
+ * block through the block table, stitch the scattered K/V together and run
+ * standard attention; GQA grouping from [mlqm] §3 (q head h uses KV head
+ * h / (num_q_heads / num_kv_heads)).  For sequence s with c = context_lens[s]:
+ *     out[s][h] = sum_t softmax_t(softmax_scale * <q[s][h], K_s[t]>) V_s[t],
+ *     K_s[t] = k_cache[block_tables[s][t / block_size]][t % block_size][h / group]
+ * over 0 <= t < c (c = 0 gives zeros).  INT8 caches are dequantised as
+ * code / scale on load.  Long contexts are cut into num_splits splits whose
+ * partial results are merged exactly through their log-sum-exp.
+ *
+ *   out           device [num_seqs][num_q_heads][head_dim], dtype q_dt.  Written.
+ *   q             device [num_seqs][num_q_heads][head_dim], dtype q_dt:
+ *                 PKV_BF16 for BF16/I8 caches; PKV_F32 or PKV_BF16 for F32 caches.
+ *   k_cache, v_cache, k_scale, v_scale  as above (scales only for PKV_I8).
+ *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past the
+ *                 sequence's last block are never read.
+ *   context_lens  device int32 [num_seqs].
+ *   max_context_len  host-side upper bound of context_lens (sizes the splits).
+ *   softmax_scale usually 1/sqrt(head_dim).
+ *   workspace     device scratch of >= pkv_workspace_size(...) bytes (may be NULL
+ *                 when that size is 0).  Overwritten; not read before written.
+ *   num_splits    0 = automatic, else the number of splits to use.
+ *   err_flag      device int or NULL (PKV_FLAG_BAD_BLOCK, _CTX_RANGE, _NEG_CTX).
+ * Output for a sequence with a bad block id covers its remaining tokens only.
+ */
+int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const void* k_cache,
+                               const void* v_cache, pkv_dtype cache_dt, const float* k_scale,
+                               const float* v_scale, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* context_lens,
+                               int max_context_len, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               float softmax_scale, void* workspace, size_t workspace_bytes,
+                               int num_splits, int* err_flag, pkv_stream_t stream);
+
+/*
+ * pkv_copy - device-to-device copy of `bytes` bytes (a multiple of 16) with a
+ * streaming kernel; used to measure the attainable HBM bandwidth in the same
+ * process as the attention kernels.  Not part of the attention path.
+ */
+int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream);
+
+/* Human-readable text for a pkv_status. */
+const char* pkv_strerror(int status);
+
+/* ABI version: (major << 16) | minor. */
+int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

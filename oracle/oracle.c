@@ -40,7 +40,7 @@
  *
  * Every floating-point step of the attention is in fp64 on the stored values
  * (fp32 inputs widened exactly; bf16 values arrive already widened to fp32,
- * which is exact).  OpenMP runs independent (sequence, head) problems in
+ * which is exact).  OpenMP runs independent (sequence, kv head) problems in
  * parallel; nothing inside one problem is reordered, blocked or fused.
  */
 #include <math.h>
@@ -137,57 +137,65 @@ int oracle_append_int8(const float* x, const int64_t* slot_mapping, int64_t num_
 
 /* ---------------------------------------------------------------- gather */
 
-/* Gather sequence s's first ctx tokens into contiguous fp64 rows
- * dst[t][num_kv_heads][head_dim], walking the block table. */
+/* Gather kv head kvh of sequence s's first ctx tokens into contiguous fp64
+ * rows dst[t][head_dim], walking the block table. */
 static int gather_f32(double* dst, const float* cache, const int32_t* table_row, int ctx,
-                      int num_kv_heads, int head_dim, int block_size, int num_blocks) {
+                      int num_kv_heads, int kvh, int head_dim, int block_size, int num_blocks) {
   const int64_t row = (int64_t)num_kv_heads * head_dim;
   for (int t = 0; t < ctx; ++t) {
     int32_t phys = table_row[t / block_size];
     if (phys < 0 || phys >= num_blocks) return ORACLE_ERR_BLOCK;
-    const float* src = cache + ((int64_t)phys * block_size + t % block_size) * row;
-    for (int64_t i = 0; i < row; ++i) dst[t * row + i] = (double)src[i];
+    const float* src = cache + ((int64_t)phys * block_size + t % block_size) * row +
+                       (int64_t)kvh * head_dim;
+    for (int i = 0; i < head_dim; ++i) dst[(int64_t)t * head_dim + i] = (double)src[i];
   }
   return ORACLE_OK;
 }
 
 /* Same walk for an INT8 cache, dequantising each value as code / scale. */
 static int gather_i8(double* dst, const int8_t* codes, const float* scale, const int32_t* table_row,
-                     int ctx, int num_kv_heads, int head_dim, int block_size, int num_blocks) {
+                     int ctx, int num_kv_heads, int kvh, int head_dim, int block_size,
+                     int num_blocks) {
   const int64_t row = (int64_t)num_kv_heads * head_dim;
   for (int t = 0; t < ctx; ++t) {
     int32_t phys = table_row[t / block_size];
     if (phys < 0 || phys >= num_blocks) return ORACLE_ERR_BLOCK;
     int off = t % block_size;
-    const int8_t* src = codes + ((int64_t)phys * block_size + off) * row;
-    for (int h = 0; h < num_kv_heads; ++h) {
-      double s = (double)scale[((int64_t)phys * num_kv_heads + h) * block_size + off];
-      for (int i = 0; i < head_dim; ++i)
-        dst[t * row + (int64_t)h * head_dim + i] = (double)src[h * head_dim + i] / s;
-    }
+    const int8_t* src = codes + ((int64_t)phys * block_size + off) * row + (int64_t)kvh * head_dim;
+    double s = (double)scale[((int64_t)phys * num_kv_heads + kvh) * block_size + off];
+    for (int i = 0; i < head_dim; ++i) dst[(int64_t)t * head_dim + i] = (double)src[i] / s;
   }
   return ORACLE_OK;
 }
 
-/* Exposed for the block-table worked example: gathers one sequence. */
+/* Exposed for the block-table worked example: gathers one sequence, all heads,
+ * into dst[t][num_kv_heads][head_dim]. */
 int oracle_gather_f32(double* dst, const float* cache, const int32_t* table_row, int ctx,
                       int num_kv_heads, int head_dim, int block_size, int num_blocks) {
   if (!dst || !cache || !table_row || ctx < 0) return ORACLE_ERR_ARG;
-  return gather_f32(dst, cache, table_row, ctx, num_kv_heads, head_dim, block_size, num_blocks);
+  double* one = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * head_dim);
+  int rc = ORACLE_OK;
+  for (int h = 0; h < num_kv_heads && rc == ORACLE_OK; ++h) {
+    rc = gather_f32(one, cache, table_row, ctx, num_kv_heads, h, head_dim, block_size, num_blocks);
+    for (int t = 0; rc == ORACLE_OK && t < ctx; ++t)
+      for (int i = 0; i < head_dim; ++i)
+        dst[((int64_t)t * num_kv_heads + h) * head_dim + i] = one[(int64_t)t * head_dim + i];
+  }
+  free(one);
+  return rc;
 }
 
 /* ---------------------------------------------------------------- attention */
 
 /* Standard attention of one q head over contiguous K/V rows (fp64).
- * q: [head_dim]; K,V: [ctx][num_kv_heads][head_dim]; reads head kvh. */
+ * q: [head_dim]; K,V: [ctx][head_dim]. */
 static void attend_one(double* out, const float* q, const double* K, const double* V, int ctx,
-                       int num_kv_heads, int kvh, int head_dim, double softmax_scale, double* z) {
-  const int64_t row = (int64_t)num_kv_heads * head_dim;
+                       int head_dim, double softmax_scale, double* z) {
   for (int i = 0; i < head_dim; ++i) out[i] = 0.0;
   if (ctx == 0) return;
   double zmax = -INFINITY;
   for (int t = 0; t < ctx; ++t) {
-    const double* k = K + t * row + (int64_t)kvh * head_dim;
+    const double* k = K + (int64_t)t * head_dim;
     double dot = 0.0;
     for (int i = 0; i < head_dim; ++i) dot += (double)q[i] * k[i];
     z[t] = softmax_scale * dot;
@@ -199,20 +207,10 @@ static void attend_one(double* out, const float* q, const double* K, const doubl
     denom += z[t];
   }
   for (int t = 0; t < ctx; ++t) {
-    const double* v = V + t * row + (int64_t)kvh * head_dim;
+    const double* v = V + (int64_t)t * head_dim;
     double p = z[t] / denom;
     for (int i = 0; i < head_dim; ++i) out[i] += p * v[i];
   }
-}
-
-/* Attention on contiguous K/V for all q heads of one sequence. */
-static void attend_seq(double* out, const float* q, const double* K, const double* V, int ctx,
-                       int num_q_heads, int num_kv_heads, int head_dim, double softmax_scale,
-                       double* z) {
-  const int group = num_q_heads / num_kv_heads;
-  for (int h = 0; h < num_q_heads; ++h)
-    attend_one(out + (int64_t)h * head_dim, q + (int64_t)h * head_dim, K, V, ctx, num_kv_heads,
-               h / group, head_dim, softmax_scale, z);
 }
 
 static int check_shapes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -228,6 +226,76 @@ static int check_shapes(int num_seqs, int num_q_heads, int num_kv_heads, int hea
   return ORACLE_OK;
 }
 
+/* One (sequence, kv head) problem: gather that head's K/V rows of the
+ * sequence, then attend for each q head h with h / group == kvh. */
+static int decode_problem(double* out, const float* q, const float* k_cache, const float* v_cache,
+                          const int8_t* k_codes, const int8_t* v_codes, const float* k_scale,
+                          const float* v_scale, const int32_t* block_tables,
+                          int max_blocks_per_seq, const int32_t* context_lens, int s, int kvh,
+                          int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                          int num_blocks, double softmax_scale) {
+  const int ctx = context_lens[s];
+  const int group = num_q_heads / num_kv_heads;
+  const size_t n = (size_t)(ctx > 0 ? ctx : 1);
+  double* K = (double*)malloc(sizeof(double) * n * head_dim);
+  double* V = (double*)malloc(sizeof(double) * n * head_dim);
+  double* z = (double*)malloc(sizeof(double) * n);
+  const int32_t* trow = block_tables + (int64_t)s * max_blocks_per_seq;
+  int e;
+  if (k_codes) {
+    e = gather_i8(K, k_codes, k_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
+                  num_blocks);
+    if (!e)
+      e = gather_i8(V, v_codes, v_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
+                    num_blocks);
+  } else {
+    e = gather_f32(K, k_cache, trow, ctx, num_kv_heads, kvh, head_dim, block_size, num_blocks);
+    if (!e)
+      e = gather_f32(V, v_cache, trow, ctx, num_kv_heads, kvh, head_dim, block_size, num_blocks);
+  }
+  if (!e) {
+    for (int h = 0; h < num_q_heads; ++h) {
+      if (h / group != kvh) continue;
+      const int64_t r = ((int64_t)s * num_q_heads + h) * head_dim;
+      attend_one(out + r, q + r, K, V, ctx, head_dim, softmax_scale, z);
+    }
+  }
+  free(K);
+  free(V);
+  free(z);
+  return e;
+}
+
+static int decode_all(double* out, const float* q, const float* k_cache, const float* v_cache,
+                      const int8_t* k_codes, const int8_t* v_codes, const float* k_scale,
+                      const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
+                      const int32_t* context_lens, int num_seqs, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      double softmax_scale, int num_threads) {
+  int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                        max_blocks_per_seq, context_lens);
+  if (rc) return rc;
+  int err = ORACLE_OK;
+  const int64_t problems = (int64_t)num_seqs * num_kv_heads;
+#ifdef _OPENMP
+  if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int64_t i = 0; i < problems; ++i) {
+    int e = decode_problem(out, q, k_cache, v_cache, k_codes, v_codes, k_scale, v_scale,
+                           block_tables, max_blocks_per_seq, context_lens, (int)(i / num_kv_heads),
+                           (int)(i % num_kv_heads), num_q_heads, num_kv_heads, head_dim,
+                           block_size, num_blocks, softmax_scale);
+    if (e) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+      err = e;
+    }
+  }
+  return err;
+}
+
 /* Paged decode over an fp32-valued cache (bf16 caches are passed widened).
  * out: [num_seqs][num_q_heads][head_dim] fp64; q: same shape, fp32-valued.
  * k_cache, v_cache: [num_blocks][block_size][num_kv_heads][head_dim].
@@ -238,38 +306,9 @@ int oracle_paged_decode_f32(double* out, const float* q, const float* k_cache,
                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                             int num_blocks, double softmax_scale, int num_threads) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return ORACLE_ERR_ARG;
-  int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                        max_blocks_per_seq, context_lens);
-  if (rc) return rc;
-  int err = ORACLE_OK;
-  const int64_t qrow = (int64_t)num_q_heads * head_dim;
-  const int64_t kvrow = (int64_t)num_kv_heads * head_dim;
-#ifdef _OPENMP
-  if (num_threads > 0) omp_set_num_threads(num_threads);
-#pragma omp parallel for schedule(dynamic, 1)
-#endif
-  for (int s = 0; s < num_seqs; ++s) {
-    int ctx = context_lens[s];
-    double* K = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * kvrow);
-    double* V = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * kvrow);
-    double* z = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1));
-    const int32_t* trow = block_tables + (int64_t)s * max_blocks_per_seq;
-    int e = gather_f32(K, k_cache, trow, ctx, num_kv_heads, head_dim, block_size, num_blocks);
-    if (!e) e = gather_f32(V, v_cache, trow, ctx, num_kv_heads, head_dim, block_size, num_blocks);
-    if (!e)
-      attend_seq(out + s * qrow, q + s * qrow, K, V, ctx, num_q_heads, num_kv_heads, head_dim,
-                 softmax_scale, z);
-    if (e) {
-#ifdef _OPENMP
-#pragma omp critical
-#endif
-      err = e;
-    }
-    free(K);
-    free(V);
-    free(z);
-  }
-  return err;
+  return decode_all(out, q, k_cache, v_cache, NULL, NULL, NULL, NULL, block_tables,
+                    max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                    head_dim, block_size, num_blocks, softmax_scale, num_threads);
 }
 
 /* Paged decode over an INT8 cache: codes [num_blocks][block_size][num_kv_heads]
@@ -283,41 +322,9 @@ int oracle_paged_decode_i8(double* out, const float* q, const int8_t* k_codes,
                            double softmax_scale, int num_threads) {
   if (!out || !q || !k_codes || !v_codes || !k_scale || !v_scale || !block_tables || !context_lens)
     return ORACLE_ERR_ARG;
-  int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                        max_blocks_per_seq, context_lens);
-  if (rc) return rc;
-  int err = ORACLE_OK;
-  const int64_t qrow = (int64_t)num_q_heads * head_dim;
-  const int64_t kvrow = (int64_t)num_kv_heads * head_dim;
-#ifdef _OPENMP
-  if (num_threads > 0) omp_set_num_threads(num_threads);
-#pragma omp parallel for schedule(dynamic, 1)
-#endif
-  for (int s = 0; s < num_seqs; ++s) {
-    int ctx = context_lens[s];
-    double* K = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * kvrow);
-    double* V = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * kvrow);
-    double* z = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1));
-    const int32_t* trow = block_tables + (int64_t)s * max_blocks_per_seq;
-    int e = gather_i8(K, k_codes, k_scale, trow, ctx, num_kv_heads, head_dim, block_size,
-                      num_blocks);
-    if (!e)
-      e = gather_i8(V, v_codes, v_scale, trow, ctx, num_kv_heads, head_dim, block_size,
-                    num_blocks);
-    if (!e)
-      attend_seq(out + s * qrow, q + s * qrow, K, V, ctx, num_q_heads, num_kv_heads, head_dim,
-                 softmax_scale, z);
-    if (e) {
-#ifdef _OPENMP
-#pragma omp critical
-#endif
-      err = e;
-    }
-    free(K);
-    free(V);
-    free(z);
-  }
-  return err;
+  return decode_all(out, q, NULL, NULL, k_codes, v_codes, k_scale, v_scale, block_tables,
+                    max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                    head_dim, block_size, num_blocks, softmax_scale, num_threads);
 }
 
 int oracle_max_threads(void) {

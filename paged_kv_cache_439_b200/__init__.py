@@ -1,1 +1,13 @@
-"""Paged-KV decode attention for B200 (sm_100a)."""
+"""Paged-KV decode attention for NVIDIA B200 (sm_100a).
+
+The kernels and their C ABI live in ``libpkv.so`` (``include/pkv.h``); this
+package is the thin Python binding plus the seeded workload generator.
+"""
+from ._native import PkvError, PKV_FLAG_BAD_BLOCK, PKV_FLAG_BAD_SLOT, PKV_FLAG_CTX_RANGE, \
+    PKV_FLAG_NEG_CTX
+from .api import (copy, decode_num_splits, kv_cache_append, paged_attention_decode,
+                  workspace_size)
+
+__all__ = ["PkvError", "kv_cache_append", "paged_attention_decode", "workspace_size",
+           "decode_num_splits", "copy", "PKV_FLAG_BAD_BLOCK", "PKV_FLAG_BAD_SLOT",
+           "PKV_FLAG_CTX_RANGE", "PKV_FLAG_NEG_CTX"]

@@ -1,0 +1,236 @@
+// C ABI of libpkv.so: argument validation, split planning, launches.
+// The declarations and their contracts are in include/pkv.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "decode.cuh"
+#include "pkv.h"
+
+namespace {
+
+constexpr int kMaxChunk = 8192;   // tokens per split (bounds the block-table slice in smem)
+constexpr int kMinChunk = 256;    // below this a split costs more than it balances
+constexpr int kTile = 16;         // tokens per tile of the decode kernels
+constexpr int kCtasPerSlot = 4;   // target CTAs per resident-CTA slot of the device
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+int log2i(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+// Smallest number of splits allowed and the automatic choice.
+int min_splits(int max_ctx) { return max_ctx <= 0 ? 1 : (max_ctx + kMaxChunk - 1) / kMaxChunk; }
+
+int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_dtype cache_dt) {
+  if (max_ctx <= 0 || num_seqs <= 0) return 1;
+  const long long units = (long long)num_seqs * num_kv_heads;
+  const long long slots = (long long)sm_count() * pkv::decode_ctas_per_sm_hint(cache_dt, head_dim);
+  long long want = (kCtasPerSlot * slots + units - 1) / units;
+  const int lo = min_splits(max_ctx);
+  const int hi = (max_ctx + kMinChunk - 1) / kMinChunk;
+  if (want > hi) want = hi;
+  if (want < lo) want = lo;
+  return (int)want;
+}
+
+// Normalises a split count: chunk = 16-aligned ceil(max_ctx / s), s = ceil(max_ctx / chunk).
+void plan(int max_ctx, int s_req, int* s_out, int* chunk_out) {
+  if (max_ctx <= 0) {
+    *s_out = 1;
+    *chunk_out = kTile;
+    return;
+  }
+  int chunk = round_up((max_ctx + s_req - 1) / s_req, kTile);
+  *chunk_out = chunk;
+  *s_out = (max_ctx + chunk - 1) / chunk;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t ws_bytes(int num_seqs, int num_q_heads, int head_dim, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = (size_t)num_seqs * num_q_heads * splits;
+  return align256(rows * head_dim * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+int map_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int pkv_version(void) { return (1 << 16) | 0; }
+
+const char* pkv_strerror(int status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_ARG: return "invalid argument (null pointer, negative size or n_q % n_kv != 0)";
+    case PKV_ERR_DTYPE: return "unsupported dtype combination";
+    case PKV_ERR_SHAPE:
+      return "unsupported shape (head_dim must be 64 or 128, block_size a power of two in "
+             "[8, 256], group in [1, 16])";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_WORKSPACE: return "workspace missing or smaller than pkv_workspace_size()";
+    case PKV_ERR_CUDA: return "CUDA runtime error";
+    case PKV_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    default: return "unknown pkv status";
+  }
+}
+
+int pkv_kv_cache_append(const void* k, const void* v, const int64_t* slot_mapping,
+                        int num_tokens, int num_kv_heads, int head_dim, pkv_dtype in_dt,
+                        void* k_cache, void* v_cache, pkv_dtype cache_dt, int num_blocks,
+                        int block_size, float* k_scale, float* v_scale, int* err_flag,
+                        pkv_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PKV_ERR_ARG;
+  if (!k_cache || !v_cache) return PKV_ERR_ARG;
+  if (num_tokens > 0 && (!k || !v || !slot_mapping)) return PKV_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
+  if (!pow2_in(block_size, 8, 256)) return PKV_ERR_SHAPE;
+  if (in_dt != PKV_F32 && in_dt != PKV_BF16) return PKV_ERR_DTYPE;
+  if (cache_dt != in_dt && cache_dt != PKV_I8) return PKV_ERR_DTYPE;
+  if (cache_dt == PKV_I8 && (!k_scale || !v_scale)) return PKV_ERR_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8) || !aligned(k_scale, 4) || !aligned(v_scale, 4) ||
+      !aligned(err_flag, 4))
+    return PKV_ERR_ALIGN;
+  if (num_tokens == 0) return PKV_OK;
+  return map_cuda(pkv::launch_append(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                     in_dt, k_cache, v_cache, cache_dt, num_blocks, block_size,
+                                     k_scale, v_scale, err_flag, (cudaStream_t)stream));
+}
+
+int pkv_decode_num_splits(int num_seqs, int num_kv_heads, int head_dim, int max_context_len,
+                          pkv_dtype cache_dt) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0) return PKV_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
+  if (cache_dt != PKV_F32 && cache_dt != PKV_BF16 && cache_dt != PKV_I8) return PKV_ERR_DTYPE;
+  int s, chunk;
+  plan(max_context_len, auto_splits(num_seqs, num_kv_heads, head_dim, max_context_len, cache_dt),
+       &s, &chunk);
+  return s;
+}
+
+size_t pkv_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                          int max_context_len, pkv_dtype cache_dt, int num_splits) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0 ||
+      num_splits < 0)
+    return 0;
+  int req = num_splits;
+  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, max_context_len, cache_dt);
+  int s, chunk;
+  plan(max_context_len, req, &s, &chunk);
+  return ws_bytes(num_seqs, num_q_heads, head_dim, s);
+}
+
+int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const void* k_cache,
+                               const void* v_cache, pkv_dtype cache_dt, const float* k_scale,
+                               const float* v_scale, const int32_t* block_tables,
+                               int max_blocks_per_seq, const int32_t* context_lens,
+                               int max_context_len, int num_seqs, int num_q_heads,
+                               int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                               float softmax_scale, void* workspace, size_t workspace_bytes,
+                               int num_splits, int* err_flag, pkv_stream_t stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || num_splits < 0)
+    return PKV_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_ARG;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_ARG;
+  if (!isfinite(softmax_scale)) return PKV_ERR_ARG;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PKV_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
+  if (!pow2_in(block_size, 8, 256)) return PKV_ERR_SHAPE;
+  if (cache_dt == PKV_BF16 || cache_dt == PKV_I8) {
+    if (q_dt != PKV_BF16) return PKV_ERR_DTYPE;
+  } else if (cache_dt == PKV_F32) {
+    if (q_dt != PKV_F32 && q_dt != PKV_BF16) return PKV_ERR_DTYPE;
+  } else {
+    return PKV_ERR_DTYPE;
+  }
+  if (cache_dt == PKV_I8 && (!k_scale || !v_scale)) return PKV_ERR_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_tables, 4) ||
+      !aligned(context_lens, 4) || !aligned(err_flag, 4) || !aligned(workspace, 16))
+    return PKV_ERR_ALIGN;
+  if (num_seqs == 0) return PKV_OK;
+  if (num_seqs > 65535) return PKV_ERR_UNSUPPORTED;  // grid y dimension
+
+  long long cap = (long long)max_blocks_per_seq * block_size;
+  const int max_ctx = (int)(max_context_len < cap ? max_context_len : cap);
+  int req = num_splits;
+  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, max_ctx, cache_dt);
+  if (req < min_splits(max_ctx)) return PKV_ERR_UNSUPPORTED;
+  int splits, chunk;
+  plan(max_ctx, req, &splits, &chunk);
+  const size_t need = ws_bytes(num_seqs, num_q_heads, head_dim, splits);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return PKV_ERR_WORKSPACE;
+
+  pkv::DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.err_flag = err_flag;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.block_size = block_size;
+  p.log2_bs = log2i(block_size);
+  p.num_blocks = num_blocks;
+  p.max_context_len = max_context_len;
+  p.chunk = chunk;
+  p.num_splits = splits;
+  p.phys_bytes = round_up((chunk / block_size + 2) * 4, 128);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.q_f32 = q_dt == PKV_F32;
+  p.out_f32 = q_dt == PKV_F32;
+  if (splits > 1) {
+    const size_t rows = (size_t)num_seqs * num_q_heads * splits;
+    p.ws_o = static_cast<float*>(workspace);
+    p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        align256(rows * head_dim * sizeof(float)));
+  } else {
+    p.ws_o = nullptr;
+    p.ws_lse = nullptr;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = pkv::launch_decode(p, cache_dt, head_dim, st);
+  if (e != cudaSuccess) return PKV_ERR_CUDA;
+  if (splits > 1) {
+    e = pkv::launch_merge(p, head_dim, st);
+    if (e != cudaSuccess) return PKV_ERR_CUDA;
+  }
+  return PKV_OK;
+}
+
+int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream) {
+  if (!dst || !src) return PKV_ERR_ARG;
+  if (bytes % 16) return PKV_ERR_ARG;
+  if (!aligned(dst, 16) || !aligned(src, 16)) return PKV_ERR_ALIGN;
+  return map_cuda(pkv::launch_copy(dst, src, bytes, sm_count(), (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Launch parameters and host entry points of the decode kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pkv.h"
+
+namespace pkv {
+
+struct DecodeParams {
+  void* out;                    // [num_seqs][num_q_heads][head_dim], bf16 or fp32
+  const void* q;                // same shape, bf16 or fp32
+  const void* k_cache;          // [num_blocks][block_size][num_kv_heads][head_dim]
+  const void* v_cache;
+  const float* k_scale;         // [num_blocks][num_kv_heads][block_size] (INT8 only)
+  const float* v_scale;
+  const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
+  const int32_t* context_lens;  // [num_seqs]
+  float* ws_o;                  // [num_seqs][num_q_heads][num_splits][head_dim]
+  float* ws_lse;                // [num_seqs][num_q_heads][num_splits] (log2 domain)
+  int* err_flag;                // may be null
+  int max_blocks_per_seq;
+  int num_seqs, num_q_heads, num_kv_heads, group;
+  int block_size, log2_bs, num_blocks;
+  int max_context_len;
+  int chunk;       // tokens per split (multiple of 16)
+  int num_splits;
+  int phys_bytes;  // shared-memory bytes reserved for the block-table slice
+  float scale_log2;  // softmax_scale * log2(e)
+  int q_f32;
+  int out_f32;
+};
+
+cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
+                          cudaStream_t st);
+cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st);
+int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim);
+
+cudaError_t launch_append(const void* k, const void* v, const int64_t* slot_mapping,
+                          int num_tokens, int num_kv_heads, int head_dim, pkv_dtype in_dt,
+                          void* k_cache, void* v_cache, pkv_dtype cache_dt, int num_blocks,
+                          int block_size, float* k_scale, float* v_scale, int* err_flag,
+                          cudaStream_t st);
+
+cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t st);
+
+}  // namespace pkv

@@ -140,7 +140,7 @@ def make_custom(name: str, context_lens: List[int], num_q_heads: int, num_kv_hea
                 input_dtype: torch.dtype = torch.bfloat16, softmax_scale: Optional[float] = None,
                 pool_factor: float = 1.2, min_pool: int = 0, shared_prefix: int = 0,
                 outlier_prob: float = 0.0, pad_entry: int = -1, extra_table_cols: int = 0,
-                randomize: bool = True) -> Workload:
+                randomize: bool = True, placement_seed: Optional[int] = None) -> Workload:
     """Builds a workload from explicit lengths.
 
     ``shared_prefix`` > 0 (a multiple of block_size) makes every sequence
@@ -169,7 +169,8 @@ def make_custom(name: str, context_lens: List[int], num_q_heads: int, num_kv_hea
     need = prefix_blocks + sum(nblk(c) - prefix_blocks for c in lens) if shared_prefix else \
         sum(nblk(c) for c in lens)
     num_blocks = max(int(math.ceil(pool_factor * need)), need, min_pool, 1)
-    alloc = BlockAllocator(num_blocks, gen if randomize else None)
+    place_gen = gen if placement_seed is None else torch.Generator().manual_seed(placement_seed)
+    alloc = BlockAllocator(num_blocks, place_gen if randomize else None)
 
     max_blocks = max([nblk(c) for c in lens] + [1]) + extra_table_cols
     tables = torch.full((B, max_blocks), pad_entry, dtype=torch.int32)

@@ -1,0 +1,121 @@
+"""The C ABI library loads, exports every symbol include/pkv.h declares, and its
+host-side argument checks reject bad calls before anything is launched.
+
+No GPU: the checks below return before any CUDA call (pointers are fake but
+never dereferenced on the host)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_439_b200 import build, _native
+    build.build()
+    return _native.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("pkv_kv_cache_append", "pkv_paged_attention_decode", "pkv_workspace_size",
+                     "pkv_decode_num_splits", "pkv_strerror", "pkv_copy", "pkv_version"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from paged_kv_cache_439_b200 import _native
+    out = subprocess.run(["nm", "-D", "--defined-only", _native.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(pkv_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(lib, n)
+    # and the binding's prototype table covers them all
+    assert set(_native.SIGNATURES) == set(_declared())
+
+
+def test_strerror_and_version(lib):
+    assert lib.pkv_strerror(0) == b"ok"
+    for s in range(-7, 0):
+        assert lib.pkv_strerror(s) and lib.pkv_strerror(s) != b"unknown pkv status"
+    assert lib.pkv_version() >> 16 == 1
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced by the host checks
+
+
+def _decode(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, q_dt=1, k=FAKE, v=FAKE, cdt=1, ks=None, vs=None, bt=FAKE,
+             maxb=4, cl=FAKE, maxctx=64, B=2, nq=8, nkv=2, d=128, bs=16, nb=10, scale=0.1,
+             ws=None, wsb=0, splits=1, err=None, stream=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode(
+        a["out"], a["q"], a["q_dt"], a["k"], a["v"], a["cdt"], a["ks"], a["vs"], a["bt"],
+        a["maxb"], a["cl"], a["maxctx"], a["B"], a["nq"], a["nkv"], a["d"], a["bs"], a["nb"],
+        a["scale"], a["ws"], a["wsb"], a["splits"], a["err"], a["stream"])
+
+
+def test_decode_argument_errors(lib):
+    assert _decode(lib, nq=6, nkv=4) == -1            # n_q % n_kv != 0
+    assert _decode(lib, out=None) == -1
+    assert _decode(lib, B=-1) == -1
+    assert _decode(lib, d=96) == -3                    # head_dim outside {64, 128}
+    assert _decode(lib, bs=12) == -3                   # not a power of two
+    assert _decode(lib, bs=512) == -3
+    assert _decode(lib, nq=34, nkv=2) == -3            # group 17 > 16
+    assert _decode(lib, cdt=1, q_dt=0) == -2           # bf16 cache needs bf16 q
+    assert _decode(lib, cdt=7) == -2
+    assert _decode(lib, cdt=2) == -1                   # int8 without scales
+    assert _decode(lib, q=FAKE + 8) == -7              # misaligned
+    assert _decode(lib, splits=2, maxctx=64) == -5     # split-K without workspace
+    assert _decode(lib, B=0) == 0                      # nothing to do
+    assert _decode(lib, scale=float("nan")) == -1
+    # each split holds at most 8192 tokens
+    assert _decode(lib, maxb=1024, maxctx=16384, splits=1) == -4
+
+
+def test_append_argument_errors(lib):
+    def call(**kw):
+        a = dict(k=FAKE, v=FAKE, sm=FAKE, T=4, nkv=2, d=64, idt=1, kc=FAKE, vc=FAKE, cdt=1, nb=4,
+                 bs=16, ks=None, vs=None, err=None)
+        a.update(kw)
+        return lib.pkv_kv_cache_append(a["k"], a["v"], a["sm"], a["T"], a["nkv"], a["d"],
+                                       a["idt"], a["kc"], a["vc"], a["cdt"], a["nb"], a["bs"],
+                                       a["ks"], a["vs"], a["err"], None)
+    assert call(T=-1) == -1
+    assert call(kc=None) == -1
+    assert call(d=80) == -3
+    assert call(bs=6) == -3
+    assert call(idt=2) == -2                  # int8 input
+    assert call(idt=0, cdt=1) == -2           # fp32 -> bf16 cache not supported
+    assert call(cdt=2) == -1                  # int8 cache without scales
+    assert call(k=FAKE + 4) == -7
+    assert call(T=0) == 0                     # empty append is a no-op
+
+
+def test_workspace_sizes(lib):
+    # one split -> no workspace; explicit splits -> o and lse per (seq, head, split)
+    assert lib.pkv_workspace_size(4, 8, 2, 128, 64, 1, 1) == 0
+    rows = 4 * 8 * 3
+    o = -(-rows * 128 * 4 // 256) * 256
+    lse = -(-rows * 4 // 256) * 256
+    assert lib.pkv_workspace_size(4, 8, 2, 128, 4000, 1, 3) == o + lse
+    # the automatic choice is consistent with pkv_decode_num_splits
+    s = lib.pkv_decode_num_splits(16, 8, 128, 32768, 1)
+    assert s >= 4   # 32768 tokens need at least 4 splits of <= 8192
+    rows = 16 * 64 * s
+    assert lib.pkv_workspace_size(16, 64, 8, 128, 32768, 1, 0) == \
+        -(-rows * 128 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
