@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-copy-probe", action="store_true")
     return ap.parse_args()
 
 
@@ -284,9 +285,11 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=dev)
 
     import paged_kv_cache_439_b200 as pkv
-    from paged_kv_cache_439_b200.workloads import make_workload
+    from paged_kv_cache_439_b200 import dist as pdist
+    from paged_kv_cache_439_b200.workloads import make_workload, workload_seed
 
-    wl = make_workload(args.workload, block_size=args.block_size)
+    wl = make_workload(args.workload, block_size=args.block_size,
+                       data_seed=pdist.replica_seed(workload_seed(args.workload), rank))
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8}[wl.cache_dtype]
     shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
     k_cache = torch.zeros(shape, dtype=tdt, device=dev)
@@ -360,13 +363,9 @@ def main():
         total_ms, call_ms, clocks = timed_region()
         remeasured = True
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-
+    max_ms = pdist.max_over_ranks(total_ms, device=dev)
     kv = wl.kv_bytes()
-    value = kv * K * world / (max_ms / 1e3) / 1e9
+    value = pdist.whole_job_rate(kv, K, world, max_ms)
     decode_ms = statistics.mean(call_ms)
     achieved = kv / (decode_ms / 1e3) / 1e9
     peak, peak_kind = measured_peak()
@@ -378,6 +377,8 @@ def main():
     # HBM copy probe in the same process (informational)
     copy_gbs = None
     try:
+        if args.no_copy_probe:
+            raise RuntimeError("skipped")
         nbytes = 2 << 30
         a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         b = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -433,11 +434,8 @@ def main():
             e2e_step()
         s1.record()
         torch.cuda.synchronize()
-        te = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
-        e2e = {"value": round(kv * K * world / (e2e_ms / 1e3) / 1e9, 2), "unit": "GB/s",
+        e2e_ms = pdist.max_over_ranks(s0.elapsed_time(s1), device=dev)
+        e2e = {"value": round(pdist.whole_job_rate(kv, K, world, e2e_ms), 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(e2e_ms / K, 4)}
 

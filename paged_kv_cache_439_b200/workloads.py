@@ -27,7 +27,8 @@ from typing import Dict, List, Optional
 
 import torch
 
-__all__ = ["BlockAllocator", "Workload", "CONFIGS", "make_workload", "make_custom"]
+__all__ = ["BlockAllocator", "Workload", "CONFIGS", "make_workload", "make_custom",
+           "workload_seed", "canonical_name"]
 
 
 class BlockAllocator:
@@ -248,12 +249,22 @@ _ALIASES = {"1": "tiny", "2": "llama2-7b-mha", "3": "llama2-70b-gqa", "4": "llam
             "5": "shared-prefix"}
 
 
+def canonical_name(name: str) -> str:
+    return _ALIASES.get(str(name), name)
+
+
+def workload_seed(name: str) -> int:
+    """Base seed of a named workload: 439_000 + its index (1-based)."""
+    return 439_000 + list(CONFIGS).index(canonical_name(name)) + 1
+
+
 def make_workload(name: str, block_size: Optional[int] = None, batch: Optional[int] = None,
-                  **kw) -> Workload:
-    """The named workload.  ``batch`` truncates the batch (for sampled checks)."""
-    name = _ALIASES.get(str(name), name)
-    idx = list(CONFIGS).index(name) + 1
-    seed = 439_000 + idx
+                  data_seed: Optional[int] = None, **kw) -> Workload:
+    """The named workload.  ``batch`` truncates the batch (for sampled checks);
+    ``data_seed`` re-draws the values (and placement) keeping every shape and
+    length of the workload."""
+    name = canonical_name(name)
+    seed = workload_seed(name)
     gen = torch.Generator().manual_seed(seed)
     if name == "tiny":
         lens = [17, 33, 64, 100]
@@ -282,4 +293,4 @@ def make_workload(name: str, block_size: Optional[int] = None, batch: Optional[i
     if batch is not None:
         lens = lens[:batch]
     wl.update(kw)
-    return make_custom(name, lens, seed=seed, **wl)
+    return make_custom(name, lens, seed=seed if data_seed is None else data_seed, **wl)

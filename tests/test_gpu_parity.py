@@ -23,7 +23,7 @@ RAGGED = [1, 2, 15, 16, 17, 31, 33, 100, 255, 257, 1000]
 
 
 def _wl(cache_dtype, nq, nkv, d, bs, lens=RAGGED, seed=11, **kw):
-    idt = torch.float32 if cache_dtype == "f32" else torch.bfloat16
+    idt = kw.pop("input_dtype", torch.float32 if cache_dtype == "f32" else torch.bfloat16)
     return make_custom(f"{cache_dtype}-{nq}-{nkv}-{d}-{bs}", lens, nq, nkv, d, bs, cache_dtype,
                        seed=seed, input_dtype=idt, **kw)
 
