@@ -25,6 +25,8 @@
 //  * simt (fp32 caches): fp32 FMA dot products, 2 lanes per token.
 #include <math_constants.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -713,13 +715,26 @@ __global__ void __launch_bounds__(HD) merge_kernel(const DecodeParams p) {
 
 namespace {
 
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel) to
+// the largest size any launch can ask for; later launches skip the runtime
+// call.  Racing first calls from several host threads both set the same value.
+constexpr int kMaxDevices = 64;
+constexpr int kSmemCeiling = 227 * 1024;
+
 template <class K>
 cudaError_t prepare(K kernel, int smem) {
-  // The attribute is per function and per device; setting it is cheap and
-  // idempotent, so it is simply set before every launch that needs it.
-  if (smem > 48 * 1024)
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  return cudaSuccess;
+  static std::atomic<bool> done[kMaxDevices];
+  if (smem <= 48 * 1024) return cudaSuccess;
+  if (smem > kSmemCeiling) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire))
+    return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCeiling);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices)
+    done[dev].store(true, std::memory_order_release);
+  return e;
 }
 
 template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>

@@ -110,6 +110,9 @@ def test_decode_block_sizes(cache_dtype, bs):
 
 def test_fp32_cache_bf16_query():
     wl = _wl("f32", 4, 2, 64, 16, input_dtype=torch.bfloat16)
+    # the fp32 cache holds the bf16 values widened exactly; q stays bf16
+    for name in ("prefill_k", "prefill_v", "new_k", "new_v"):
+        setattr(wl, name, getattr(wl, name).float())
     g = GpuCache(wl).fill()
     ref = OracleCache(wl).fill().decode()
     out = g.decode()
