@@ -717,23 +717,28 @@ namespace {
 
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel) to
 // the largest size any launch can ask for; later launches skip the runtime
-// call.  Racing first calls from several host threads both set the same value.
+// call.  The flag array is per kernel (the kernel is the template argument).
+// Racing first calls from several host threads both set the same value.
 constexpr int kMaxDevices = 64;
-constexpr int kSmemCeiling = 227 * 1024;
 
-template <class K>
-cudaError_t prepare(K kernel, int smem) {
-  static std::atomic<bool> done[kMaxDevices];
+template <auto Kernel>
+cudaError_t prepare(int smem) {
+  static std::atomic<int> limit[kMaxDevices];  // raised limit per device, 0 = not yet
   if (smem <= 48 * 1024) return cudaSuccess;
-  if (smem > kSmemCeiling) return cudaErrorInvalidValue;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire))
-    return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemCeiling);
-  if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices)
-    done[dev].store(true, std::memory_order_release);
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached) {
+    const int l = limit[dev].load(std::memory_order_acquire);
+    if (l > 0) return smem <= l ? cudaSuccess : cudaErrorInvalidValue;
+  }
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  if (smem > optin) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && cached) limit[dev].store(optin, std::memory_order_release);
   return e;
 }
 
@@ -749,9 +754,9 @@ int mma_smem(const DecodeParams& p) {
 
 template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  auto k = decode_mma_kernel<HD, I8, NT, NWARPS, NSTAGES>;
+  constexpr auto k = decode_mma_kernel<HD, I8, NT, NWARPS, NSTAGES>;
   const int smem = mma_smem<HD, I8, NT, NWARPS, NSTAGES>(p);
-  cudaError_t e = prepare(k, smem);
+  cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
   return cudaGetLastError();
@@ -764,8 +769,8 @@ cudaError_t launch_simt(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int GP = 16;
   constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
   const int smem = p.phys_bytes + GP * HD * 4 + (RING > COMB ? RING : COMB);
-  auto k = decode_simt_kernel<HD, NWARPS, NSTAGES>;
-  cudaError_t e = prepare(k, smem);
+  constexpr auto k = decode_simt_kernel<HD, NWARPS, NSTAGES>;
+  cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
   return cudaGetLastError();
