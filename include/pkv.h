@@ -51,7 +51,8 @@ typedef enum {
   PKV_ERR_UNSUPPORTED = -4, /* no kernel for this configuration */
   PKV_ERR_WORKSPACE = -5,   /* split-K needs a workspace of pkv_workspace_size() bytes */
   PKV_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
-  PKV_ERR_ALIGN = -7        /* a device pointer is not 16-byte aligned */
+  PKV_ERR_ALIGN = -7,       /* a device pointer is not 16-byte aligned */
+  PKV_ERR_SCRATCH_LIMIT = -8 /* split-K scratch would exceed PKV_NOALLOC_SCRATCH_BYTES */
 } pkv_status;
 
 /* Bits written into *err_flag by the kernels. */
@@ -150,6 +151,39 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
  * process as the attention kernels.  Not part of the attention path.
  */
 int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream);
+
+/* Bytes of the fixed device scratch behind pkv_paged_attention_decode_noalloc. */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * pkv_paged_attention_decode_noalloc - pkv_paged_attention_decode for callers
+ * that cannot allocate device memory.  The pages have no counterpart for this
+ * call; it exists for callers such as code embedded in a host runtime that owns
+ * every device allocation and gives its plugins no allocator or workspace.
+ *
+ * Arguments, layouts and results are those of pkv_paged_attention_decode minus
+ * `workspace` and `workspace_bytes`: the split-K scratch lives in one fixed
+ * device array of PKV_NOALLOC_SCRATCH_BYTES (16 MiB) inside the library, held
+ * on every GPU that loads the library until the process exits.
+ *   - Returns PKV_ERR_SCRATCH_LIMIT, before any launch, when the scratch the
+ *     call needs (pkv_workspace_size for the same shape and num_splits) is
+ *     larger than that array.
+ *   - Every call shares the array: calls whose kernels overlap on the GPU
+ *     (e.g. on different streams) race and must be serialised by the caller.
+ *     Nothing in the array has to start at zero.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+int pkv_paged_attention_decode_noalloc(void* out, const void* q, pkv_dtype q_dt,
+                                       const void* k_cache, const void* v_cache,
+                                       pkv_dtype cache_dt, const float* k_scale,
+                                       const float* v_scale, const int32_t* block_tables,
+                                       int max_blocks_per_seq, const int32_t* context_lens,
+                                       int max_context_len, int num_seqs, int num_q_heads,
+                                       int num_kv_heads, int head_dim, int block_size,
+                                       int num_blocks, float softmax_scale, int num_splits,
+                                       int* err_flag, pkv_stream_t stream);
 
 /* Human-readable text for a pkv_status. */
 const char* pkv_strerror(int status);

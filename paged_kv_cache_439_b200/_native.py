@@ -18,6 +18,9 @@ PKV_FLAG_BAD_SLOT = 2
 PKV_FLAG_CTX_RANGE = 4
 PKV_FLAG_NEG_CTX = 8
 
+PKV_ERR_SCRATCH_LIMIT = -8
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
 # exported symbol -> (restype, argtypes); mirrors include/pkv.h
 _vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
 SIGNATURES = {
@@ -27,6 +30,9 @@ SIGNATURES = {
     "pkv_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "pkv_paged_attention_decode": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _i,
                                         _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _i, _vp, _vp]),
+    "pkv_paged_attention_decode_noalloc": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i,
+                                                _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
+                                                _vp]),
     "pkv_copy": (_i, [_vp, _vp, _sz, _vp]),
     "pkv_strerror": (ctypes.c_char_p, [_i]),
     "pkv_version": (_i, []),

@@ -114,6 +114,42 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     return out
 
 
+def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor,
+                                   v_cache: torch.Tensor, block_tables: torch.Tensor,
+                                   context_lens: torch.Tensor,
+                                   softmax_scale: Optional[float] = None,
+                                   k_scale: Optional[torch.Tensor] = None,
+                                   v_scale: Optional[torch.Tensor] = None,
+                                   max_context_len: Optional[int] = None,
+                                   out: Optional[torch.Tensor] = None, num_splits: int = 0,
+                                   err_flag: Optional[torch.Tensor] = None,
+                                   stream=None) -> torch.Tensor:
+    """paged_attention_decode for callers that cannot allocate device memory.
+
+    The split-K scratch is the library's fixed 16 MiB device array, so nothing
+    is allocated for it; shapes that need more raise PkvError (status -8).
+    Calls that overlap on the GPU share that array and race.  ``out`` should be
+    passed by such callers (it is only allocated here when omitted).
+    """
+    B, nq, d = q.shape
+    nb, bs, nkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    if out is None:
+        out = torch.empty_like(q)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    rc = N.lib().pkv_paged_attention_decode_noalloc(
+        _ptr(out), _ptr(q), _dt(q), _ptr(k_cache), _ptr(v_cache), _dt(k_cache), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_tables), maxb, _ptr(context_lens), max_context_len, B, nq, nkv,
+        d, bs, nb, float(softmax_scale), num_splits, _ptr(err_flag), _stream(stream))
+    N.check(rc, "pkv_paged_attention_decode_noalloc")
+    return out
+
+
 def copy(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
     """Streaming device copy (HBM bandwidth probe)."""
     nbytes = src.numel() * src.element_size()
