@@ -124,7 +124,8 @@ size_t pkv_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int h
  *   out           device [num_seqs][num_q_heads][head_dim], dtype q_dt.  Written.
  *   q             device [num_seqs][num_q_heads][head_dim], dtype q_dt:
  *                 PKV_BF16 for BF16/I8 caches; PKV_F32 or PKV_BF16 for F32 caches.
- *   k_cache, v_cache, k_scale, v_scale  as above (scales only for PKV_I8).
+ *   k_cache, v_cache, k_scale, v_scale  as above (scales only for PKV_I8; the
+ *                 scale arrays must be 16-byte aligned here).
  *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past the
  *                 sequence's last block are never read.
  *   context_lens  device int32 [num_seqs].

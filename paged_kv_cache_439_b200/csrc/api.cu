@@ -37,13 +37,33 @@ int sm_count() {
 // Smallest number of splits allowed and the automatic choice.
 int min_splits(int max_ctx) { return max_ctx <= 0 ? 1 : (max_ctx + kMaxChunk - 1) / kMaxChunk; }
 
+// Automatic split count.  With U = num_seqs * num_kv_heads (sequence, head)
+// units and R CTAs resident on the device at once:
+//  * U >= R / 2: every unit already has a CTA in the first wave, so splitting
+//    only adds partial results to merge.  Keep S = 1 unless the last wave would
+//    run under half full with fewer than two waves in total, then take the
+//    smallest S that fixes that.
+//  * U < R / 2 (few, long sequences): cut the context so that about four CTAs
+//    per resident slot exist, which also evens out unequal context lengths;
+//    no split shorter than kMinChunk tokens.
 int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_dtype cache_dt) {
   if (max_ctx <= 0 || num_seqs <= 0) return 1;
   const long long units = (long long)num_seqs * num_kv_heads;
   const long long slots = (long long)sm_count() * pkv::decode_ctas_per_sm_hint(cache_dt, head_dim);
-  long long want = (kCtasPerSlot * slots + units - 1) / units;
   const int lo = min_splits(max_ctx);
   const int hi = (max_ctx + kMinChunk - 1) / kMinChunk;
+  long long want;
+  if (2 * units >= slots) {
+    want = 1;
+    for (int s = 1; s <= 8; ++s) {
+      const long long ctas = units * s;
+      const long long full_waves = ctas / slots, rest = ctas % slots;
+      want = s;
+      if (full_waves >= 2 || rest == 0 || 2 * rest >= slots) break;
+    }
+  } else {
+    want = (kCtasPerSlot * slots + units - 1) / units;
+  }
   if (want > hi) want = hi;
   if (want < lo) want = lo;
   return (int)want;
@@ -168,8 +188,9 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
     return PKV_ERR_DTYPE;
   }
   if (cache_dt == PKV_I8 && (!k_scale || !v_scale)) return PKV_ERR_ARG;
+  // INT8 scale rows are fetched with bulk copies, which need 16-byte alignment
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(block_tables, 4) ||
+      !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(block_tables, 4) ||
       !aligned(context_lens, 4) || !aligned(err_flag, 4) || !aligned(workspace, 16))
     return PKV_ERR_ALIGN;
   if (num_seqs == 0) return PKV_OK;

@@ -24,6 +24,28 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int s
                : "memory");
 }
 
+// cp_async_16 whose destination address is computed from `dep` inside the asm
+// block, so the copy cannot issue before the instructions producing `dep` have
+// their inputs (used to refill a stage only after every ldmatrix that read it
+// has returned its data).
+__device__ __forceinline__ void cp_async_16_after(uint32_t dst, const void* src, int src_bytes,
+                                                  uint32_t dep) {
+  asm volatile(
+      "{\n .reg .b32 z;\n and.b32 z, %3, 0;\n add.u32 z, z, %0;\n"
+      " cp.async.cg.shared.global [z], [%1], 16, %2;\n}\n" ::"r"(dst),
+      "l"(src), "r"(src_bytes), "r"(dep)
+      : "memory");
+}
+
+__device__ __forceinline__ void cp_async_4_after(uint32_t dst, const void* src, int src_bytes,
+                                                 uint32_t dep) {
+  asm volatile(
+      "{\n .reg .b32 z;\n and.b32 z, %3, 0;\n add.u32 z, z, %0;\n"
+      " cp.async.ca.shared.global [z], [%1], 4, %2;\n}\n" ::"r"(dst),
+      "l"(src), "r"(src_bytes), "r"(dep)
+      : "memory");
+}
+
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, int src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(dst), "l"(src),
                "r"(src_bytes)
@@ -103,20 +125,27 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Two signed bytes of `biased` (already XOR-ed with 0x80808080, so each byte is
-// b + 128) -> two exact fp16 values b.  0x64uu is the fp16 number 1024 + u;
-// subtracting 1152 = 1024 + 128 leaves b exactly.  SEL picks the two bytes.
+// Two bytes of `biased` (each b + 128) -> two exact fp16 values b + 1152
+// (0x64uu is 1024 + u).  The caller removes the constant 1152 analytically.
 template <uint32_t SEL>
-__device__ __forceinline__ uint32_t i8pair_to_f16x2(uint32_t biased) {
-  uint32_t h = prmt(biased, 0x64646464u, SEL);
-  const uint32_t k1152 = 0x64806480u;
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r) : "r"(h), "r"(k1152));
-  return r;
+__device__ __forceinline__ uint32_t i8pair_to_f16x2_biased(uint32_t biased) {
+  return prmt(biased, 0x64646464u, SEL);
+}
+
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void set_flag(int* err, int bit) {
   if (err) atomicOr(err, bit);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 }  // namespace pkv

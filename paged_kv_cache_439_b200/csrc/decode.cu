@@ -7,25 +7,22 @@
 //
 // Work decomposition: one CTA per (kv_head, sequence, context split).  All
 // `group` query heads that share a KV head live in the same CTA, so each K/V
-// byte is read from HBM once.  Inside a CTA every warp owns an interleaved
-// subset of 16-token tiles and streams them through its own cp.async ring in
-// shared memory (16-byte coalesced row segments, zero-fill for masked rows),
-// keeps an fp32 online-softmax state in registers, and the warps' states are
-// merged through shared memory at the end.  With one split the CTA writes the
-// output; otherwise it writes a normalised partial (o, log2-sum-exp) to the
-// workspace and `merge_kernel` combines the splits.
+// byte is read from HBM once.  Tiles are 16 tokens.  Each warp keeps an fp32
+// online-softmax state in registers; the warps' states are merged through
+// shared memory at the end.  With one split the CTA writes the output;
+// otherwise it writes a normalised partial (o, log2-sum-exp) to the workspace
+// and `merge_kernel` combines the splits.
 //
-// Two tile engines:
-//  * mma (bf16 and int8 caches): scores S^T = K * Q^T and the update
-//    O^T += V^T * P^T run on mma.sync m16n8k16 with fp32 accumulation, 16
-//    tokens x 8 heads per instruction.  P is split into hi + lo halves so the
-//    probabilities keep ~16 significant bits.  INT8 codes are converted to
-//    exact fp16 values in registers and the per-token scales are applied to the
-//    fp32 scores (K) and to P (V).
-//  * simt (fp32 caches): fp32 FMA dot products, 2 lanes per token.
+// Two engines:
+//  * mma (bf16 and int8 caches): per-warp cp.async stage rings; each stage is
+//    read into registers as soon as it lands and refilled at once; scores and
+//    the PV update run on mma.sync m16n8k16 with fp32 accumulation.
+//  * simt (fp32 caches): per-warp cp.async rings, fp32 FMA dot products, two
+//    lanes per token.
 #include <math_constants.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -220,19 +217,135 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
   }
 }
 
+
 // ---------------------------------------------------------------------------
 // mma engine: bf16 or int8 caches, q in bf16.
+//
+// Each warp streams its own interleaved 16-token tiles (the warp's tile i is
+// CTA tile warp + i * NWARPS) through a ring of NSTAGES cp.async stages.  As
+// soon as a stage lands it is read into registers with ldmatrix and refilled
+// with the warp's tile i + NSTAGES, so NSTAGES tiles per warp stay in flight
+// while the math runs from registers.  The refill is issued through an asm
+// block that depends on every loaded register, so it cannot overtake the
+// reads of the stage it overwrites.
+//
+// Tile math: scores S^T = K * Q^T and the update O^T += V^T * P^T on
+// mma.sync m16n8k16 with fp32 accumulation (16 tokens x 8 q heads per
+// instruction).  P is split into hi + lo halves so the probabilities keep ~16
+// significant bits.  INT8 codes become exact fp16 values in registers; the
+// per-token scales multiply the fp32 scores (K) and P (V).  The codes reach the
+// tensor core as the exact fp16 values code + 1152 (one byte permute per pair,
+// no subtraction); the constant is removed from the fp32 results: 1152 *
+// sum_d q[h][d] from every score, 1152 * sum_t P[t][h] from the output.
+
+#ifndef PKV_MMA_WARPS
+#define PKV_MMA_WARPS 4
+#endif
+#ifndef PKV_BF16_STAGES
+#define PKV_BF16_STAGES 2
+#endif
+#ifndef PKV_I8_STAGES
+#define PKV_I8_STAGES 3
+#endif
+
+template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
+struct MmaCfg {
+  static constexpr int ELEM = I8 ? 1 : 2;
+  static constexpr int ROWB = HD * ELEM;        // bytes of one token row of one head
+  static constexpr int CH = ROWB / 16;          // 16-byte chunks per row: 4, 8 or 16
+  static constexpr int RSTEP = kWarp / CH;      // rows one warp-wide copy covers
+  static constexpr int PER_LANE = 16 / RSTEP;   // copies per lane per K (or V) tile
+  static constexpr int TILE = 16 * ROWB;
+  static constexpr int STAGE = 2 * TILE + (I8 ? 128 : 0);
+  static constexpr int RING = NWARPS * NSTAGES * STAGE;
+  static constexpr int GP = NT * 8;
+  static constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
+  static constexpr int BODY = RING > COMB ? RING : COMB;
+  static_assert(CH == 4 || CH == 8 || CH == 16, "rows of 64, 128 or 256 bytes");
+};
+
+// Issues the copies of one 16-token tile (K, V and, for INT8, the 16 per-token
+// scales) into a stage, as one commit group.  Full tiles inside one block take
+// the fast path: one block-table lookup and per-lane offsets fixed for the
+// whole kernel.  Rows outside the sequence or in a bad block are zero-filled.
+// With AFTER, every copy waits for `dep` (see cp_async_16_after).
+template <class Cfg, bool AFTER>
+__device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup& c,
+                                           const int* s_phys, int tile_t0, uint32_t k_st,
+                                           uint32_t v_st, uint32_t sc_st, int lane,
+                                           const uint32_t (&soff)[Cfg::PER_LANE],
+                                           size_t lane_goff, int lane_row, uint32_t dep) {
+  const uint8_t* kb = static_cast<const uint8_t*>(p.k_cache);
+  const uint8_t* vb = static_cast<const uint8_t*>(p.v_cache);
+  const size_t tok_stride = (size_t)p.num_kv_heads * Cfg::ROWB;
+  const int bs = p.block_size;
+  if (bs >= 16 && tile_t0 + 16 <= c.t_end) {
+    const int phys = s_phys[(tile_t0 >> p.log2_bs) - c.blk0];
+    const int n = phys >= 0 ? 16 : 0;
+    const size_t base =
+        phys >= 0 ? ((size_t)phys * bs + (tile_t0 & (bs - 1))) * tok_stride + lane_goff : 0;
+#pragma unroll
+    for (int i = 0; i < Cfg::PER_LANE; ++i) {
+      const size_t off = phys >= 0 ? base + (size_t)i * Cfg::RSTEP * tok_stride : 0;
+      if constexpr (AFTER) {
+        cp_async_16_after(k_st + soff[i], kb + off, n, dep);
+        cp_async_16_after(v_st + soff[i], vb + off, n, dep);
+      } else {
+        cp_async_16(k_st + soff[i], kb + off, n);
+        cp_async_16(v_st + soff[i], vb + off, n);
+      }
+    }
+  } else {
+    const size_t lane_col = lane_goff - (size_t)lane_row * tok_stride;  // head + chunk offset
+#pragma unroll
+    for (int i = 0; i < Cfg::PER_LANE; ++i) {
+      const int row = lane_row + i * Cfg::RSTEP;
+      const int t = tile_t0 + row;
+      const int phys = phys_of(p, c, s_phys, t);
+      size_t off = 0;
+      int n = 0;
+      if (phys >= 0) {
+        off = ((size_t)phys * bs + (t & (bs - 1))) * tok_stride + lane_col;
+        n = 16;
+      }
+      if constexpr (AFTER) {
+        cp_async_16_after(k_st + soff[i], kb + off, n, dep);
+        cp_async_16_after(v_st + soff[i], vb + off, n, dep);
+      } else {
+        cp_async_16(k_st + soff[i], kb + off, n);
+        cp_async_16(v_st + soff[i], vb + off, n);
+      }
+    }
+  }
+  if constexpr (Cfg::ELEM == 1) {
+    const int row = lane & 15;
+    const int t = tile_t0 + row;
+    const int phys = phys_of(p, c, s_phys, t);
+    const float* src = (lane < 16) ? p.k_scale : p.v_scale;
+    size_t off = 0;
+    int n = 0;
+    if (phys >= 0) {
+      off = ((size_t)phys * p.num_kv_heads + c.kvh) * bs + (t & (bs - 1));
+      n = 4;
+    }
+    if constexpr (AFTER)
+      cp_async_4_after(sc_st + 4 * lane, src + off, n, dep);
+    else
+      cp_async_4(sc_st + 4 * lane, src + off, n);
+  }
+  cp_async_commit();
+}
+
 template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_mma_kernel(const DecodeParams p) {
-  constexpr int ELEM = I8 ? 1 : 2;
-  constexpr int ROWB = HD * ELEM;
-  constexpr int CH = ROWB / 16;
-  constexpr int TILE_B = 16 * ROWB;
-  constexpr int STAGE_B = 2 * TILE_B + (I8 ? 128 : 0);
-  constexpr int KS = HD / 16;  // k-steps of the score mma
-  constexpr int MT = HD / 16;  // m-tiles (16 head-dim rows) of the PV mma
-  constexpr int GP = NT * 8;
+  using Cfg = MmaCfg<HD, I8, NT, NWARPS, NSTAGES>;
+  constexpr int KS = HD / 16;           // k-steps of the score mma
+  constexpr int MT = HD / 16;           // m-tiles (16 head-dim rows) of the PV mma
+  constexpr int KA = I8 ? KS / 2 : KS;  // ldmatrix.x4 per K tile
+  constexpr int VA = I8 ? MT / 2 : MT;  // ldmatrix.x4 per V tile
+  constexpr int GP = Cfg::GP;
+  constexpr int CH = Cfg::CH;
 
   extern __shared__ __align__(128) uint8_t smem[];
   int* s_phys = reinterpret_cast<int*>(smem);
@@ -278,14 +391,34 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     }
   }
 
+  // INT8: the tensor core sees code + 1152 instead of code (see
+  // i8pair_to_f16x2_biased), so every score carries 1152 * sum_d q[h][d]; qbias
+  // holds that term for this thread's two head columns 2*t4 and 2*t4 + 1.
+  float qbias[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    float mine = 0.f;  // partial sum over this lane's k-slots of head nt*8 + g
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const float2 a = unpack_f16(qf[ks][nt][0]), b = unpack_f16(qf[ks][nt][1]);
+      mine += (a.x + a.y) + (b.x + b.y);
+    }
+    mine += __shfl_xor_sync(0xffffffffu, mine, 1);
+    mine += __shfl_xor_sync(0xffffffffu, mine, 2);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      qbias[nt][j] = I8 ? 1152.f * __shfl_sync(0xffffffffu, mine, (2 * t4 + j) * 4) : 0.f;
+  }
+
   float o[MT][NT][4];
-  float m_run[NT][2], l_run[NT][2];
+  float m_run[NT][2], l_run[NT][2], p_run[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       m_run[nt][j] = -CUDART_INF_F;
       l_run[nt][j] = 0.f;
+      p_run[nt][j] = 0.f;  // INT8: sum of the P fed to the PV mma (for its 1152 bias)
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
@@ -293,127 +426,172 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       for (int j = 0; j < 4; ++j) o[mt][nt][j] = 0.f;
   }
 
-  uint8_t* my_ring = ring + (size_t)warp * NSTAGES * STAGE_B;
-  const int ntiles = (c.t_end - c.t_begin + 15) >> 4;
-  const int my_n = (warp < ntiles) ? (ntiles - warp + NWARPS - 1) / NWARPS : 0;
-
-  auto stage_k = [&](int s) { return my_ring + (size_t)s * STAGE_B; };
-  auto stage_v = [&](int s) { return my_ring + (size_t)s * STAGE_B + TILE_B; };
-  auto stage_sc = [&](int s) {
-    return reinterpret_cast<float*>(my_ring + (size_t)s * STAGE_B + 2 * TILE_B);
-  };
-
+  // Per-lane copy geometry: lane copies chunk lane % CH of rows
+  // lane / CH + i * RSTEP; its shared-memory offsets are fixed.
+  const int lane_row = lane / CH, lane_ch = lane % CH;
+  uint32_t soff[Cfg::PER_LANE];
 #pragma unroll
-  for (int i = 0; i < NSTAGES - 1; ++i) {
-    if (i < my_n)
-      load_tile<HD, ELEM, I8>(p, c, s_phys, c.t_begin + (warp + i * NWARPS) * 16, stage_k(i),
-                              stage_v(i), stage_sc(i), lane);
-    else
-      cp_async_commit();
-  }
+  for (int i = 0; i < Cfg::PER_LANE; ++i)
+    soff[i] = (uint32_t)swz<CH>(lane_row + i * Cfg::RSTEP, lane_ch) * 16;
+  const size_t tok_stride = (size_t)p.num_kv_heads * Cfg::ROWB;
+  const size_t lane_goff =
+      (size_t)lane_row * tok_stride + (size_t)c.kvh * Cfg::ROWB + (size_t)lane_ch * 16;
 
   // ldmatrix lane addressing: matrix j = lane/8 supplies its row lane%8.
   const int lm_row_a = (lane & 7) + ((lane >> 3) & 1) * 8;  // j: rows 0-7, 8-15, 0-7, 8-15
   const int lm_ch_a = lane >> 4;                            //    chunk +0, +0, +1, +1
   const int lm_row_v = (lane & 7) + ((lane >> 4) & 1) * 8;  // j: rows 0-7, 0-7, 8-15, 8-15
   const int lm_ch_v = (lane >> 3) & 1;                      //    chunk +0, +1, +0, +1
+  uint32_t koff[KA], voff[VA];
+#pragma unroll
+  for (int i = 0; i < KA; ++i) koff[i] = (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16;
+#pragma unroll
+  for (int i = 0; i < VA; ++i)
+    voff[i] = I8 ? (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16
+                 : (uint32_t)swz<CH>(lm_row_v, 2 * i + lm_ch_v) * 16;
+
+  const uint32_t my_ring = smem_u32(ring) + (uint32_t)(warp * NSTAGES * Cfg::STAGE);
+  const int ntiles = (c.t_end - c.t_begin + 15) >> 4;
+  const int my_n = (warp < ntiles) ? (ntiles - warp + NWARPS - 1) / NWARPS : 0;
+
+#pragma unroll
+  for (int i = 0; i < NSTAGES; ++i) {
+    const uint32_t st = my_ring + (uint32_t)(i * Cfg::STAGE);
+    if (i < my_n)
+      issue_tile<Cfg, false>(p, c, s_phys, c.t_begin + (warp + i * NWARPS) * 16, st,
+                             st + Cfg::TILE, st + 2 * Cfg::TILE, lane, soff, lane_goff, lane_row,
+                             0u);
+    else
+      cp_async_commit();
+  }
 
   for (int i = 0; i < my_n; ++i) {
+    cp_async_wait<NSTAGES - 1>();
+    __syncwarp();
+    const uint32_t kS = my_ring + (uint32_t)((i % NSTAGES) * Cfg::STAGE);
+    const uint32_t vS = kS + Cfg::TILE;
+    const int tile_t0 = c.t_begin + (warp + i * NWARPS) * 16;
+
+    // ---- read the stage into registers
+    uint32_t kf[KA][4], vf[VA][4];
+#pragma unroll
+    for (int a = 0; a < KA; ++a) ldmatrix_x4(kS + koff[a], kf[a][0], kf[a][1], kf[a][2], kf[a][3]);
+#pragma unroll
+    for (int a = 0; a < VA; ++a)
+      ldmatrix_x4_trans(vS + voff[a], vf[a][0], vf[a][1], vf[a][2], vf[a][3]);
+    float ska = 0.f, skb = 0.f, sva = 0.f, svb = 0.f;
+    uint32_t dep = 0;
+    if constexpr (I8) {
+      float mine;
+      asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(mine) : "r"(vS + Cfg::TILE + 4 * lane));
+      ska = __shfl_sync(0xffffffffu, mine, g);
+      skb = __shfl_sync(0xffffffffu, mine, g + 8);
+      sva = __shfl_sync(0xffffffffu, mine, 16 + g);
+      svb = __shfl_sync(0xffffffffu, mine, 24 + g);
+      dep = __float_as_uint(mine);
+    }
+#pragma unroll
+    for (int a = 0; a < KA; ++a) dep ^= kf[a][0] ^ kf[a][1] ^ kf[a][2] ^ kf[a][3];
+#pragma unroll
+    for (int a = 0; a < VA; ++a) dep ^= vf[a][0] ^ vf[a][1] ^ vf[a][2] ^ vf[a][3];
+    const uint32_t mask =
+        __ballot_sync(0xffffffffu, phys_of(p, c, s_phys, tile_t0 + (lane & 15)) >= 0) & 0xFFFFu;
+
+    // ---- refill the stage with this warp's tile i + NSTAGES
     {
-      const int ii = i + NSTAGES - 1;
+      const int ii = i + NSTAGES;
       if (ii < my_n)
-        load_tile<HD, ELEM, I8>(p, c, s_phys, c.t_begin + (warp + ii * NWARPS) * 16,
-                                stage_k(ii % NSTAGES), stage_v(ii % NSTAGES),
-                                stage_sc(ii % NSTAGES), lane);
+        issue_tile<Cfg, true>(p, c, s_phys, c.t_begin + (warp + ii * NWARPS) * 16, kS, vS,
+                              vS + Cfg::TILE, lane, soff, lane_goff, lane_row, dep);
       else
         cp_async_commit();
     }
-    cp_async_wait<NSTAGES - 1>();
-    __syncwarp();
+    if (mask == 0u) continue;
 
-    const int st = i % NSTAGES;
-    const uint32_t kS = smem_u32(stage_k(st));
-    const uint32_t vS = smem_u32(stage_v(st));
-    const float* sc = stage_sc(st);
-    const int tile_t0 = c.t_begin + (warp + i * NWARPS) * 16;
-
-    // ---- scores S^T[token][head] = K * Q^T
-    float acc[NT][4];
+    // ---- scores S^T[token][head] = K * Q^T (two accumulator chains)
+    float acc[NT][4], acc2[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[nt][j] = 0.f;
+      for (int q = 0; q < 4; ++q) acc[nt][q] = acc2[nt][q] = 0.f;
     if constexpr (!I8) {
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4(kS + swz<CH>(lm_row_a, 2 * ks + lm_ch_a) * 16, a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          mma_bf16(acc[nt], a0, a1, a2, a3, qf[ks][nt][0], qf[ks][nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if (ks & 1)
+            mma_bf16(acc2[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
+                     qf[ks][nt][1]);
+          else
+            mma_bf16(acc[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
+                     qf[ks][nt][1]);
+        }
       }
     } else {
 #pragma unroll
       for (int kp = 0; kp < KS / 2; ++kp) {
-        uint32_t r0, r1, r2, r3;  // (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1)
-        ldmatrix_x4(kS + swz<CH>(lm_row_a, 2 * kp + lm_ch_a) * 16, r0, r1, r2, r3);
-        const uint32_t top[2] = {r0 ^ 0x80808080u, r2 ^ 0x80808080u};
-        const uint32_t bot[2] = {r1 ^ 0x80808080u, r3 ^ 0x80808080u};
+        // kf[kp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1)
+        const uint32_t top[2] = {kf[kp][0] ^ 0x80808080u, kf[kp][2] ^ 0x80808080u};
+        const uint32_t bot[2] = {kf[kp][1] ^ 0x80808080u, kf[kp][3] ^ 0x80808080u};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = i8pair_to_f16x2<0x4140>(top[h]);
-          const uint32_t a2 = i8pair_to_f16x2<0x4342>(top[h]);
-          const uint32_t a1 = i8pair_to_f16x2<0x4140>(bot[h]);
-          const uint32_t a3 = i8pair_to_f16x2<0x4342>(bot[h]);
+          const uint32_t a0 = i8pair_to_f16x2_biased<0x4140>(top[h]);
+          const uint32_t a2 = i8pair_to_f16x2_biased<0x4342>(top[h]);
+          const uint32_t a1 = i8pair_to_f16x2_biased<0x4140>(bot[h]);
+          const uint32_t a3 = i8pair_to_f16x2_biased<0x4342>(bot[h]);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_f16(acc[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
+          for (int nt = 0; nt < NT; ++nt) {
+            if (h)
+              mma_f16(acc2[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
+            else
+              mma_f16(acc[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
+          }
         }
       }
     }
 
-    // ---- mask, scale, online softmax (this thread: tokens g, g+8; heads 2t4, 2t4+1)
-    const int ta = tile_t0 + g, tb = tile_t0 + g + 8;
-    const bool va = phys_of(p, c, s_phys, ta) >= 0;
-    const bool vb = phys_of(p, c, s_phys, tb) >= 0;
+    // ---- mask, scale, online softmax (tokens g, g+8; heads 2t4, 2t4+1)
+    const bool va = (mask >> g) & 1u, vb = (mask >> (g + 8)) & 1u;
     float fa = p.scale_log2, fb = p.scale_log2;
     float pva = 1.f, pvb = 1.f;
     if constexpr (I8) {
-      fa = va ? fa / sc[g] : 0.f;
-      fb = vb ? fb / sc[g + 8] : 0.f;
-      pva = va ? 1.f / sc[16 + g] : 0.f;
-      pvb = vb ? 1.f / sc[16 + g + 8] : 0.f;
+      fa = va ? fa * fast_rcp(ska) : 0.f;
+      fb = vb ? fb * fast_rcp(skb) : 0.f;
+      pva = va ? fast_rcp(sva) : 0.f;
+      pvb = vb ? fast_rcp(svb) : 0.f;
     }
     uint32_t bh[NT][2], bl[NT][2];
+    float alpha[NT][2];
+    bool rescale = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      float s[4];
-      s[0] = va ? acc[nt][0] * fa : -CUDART_INF_F;
-      s[1] = va ? acc[nt][1] * fa : -CUDART_INF_F;
-      s[2] = vb ? acc[nt][2] * fb : -CUDART_INF_F;
-      s[3] = vb ? acc[nt][3] * fb : -CUDART_INF_F;
+      float sv[4];
+      sv[0] = va ? ((acc[nt][0] + acc2[nt][0]) - qbias[nt][0]) * fa : -CUDART_INF_F;
+      sv[1] = va ? ((acc[nt][1] + acc2[nt][1]) - qbias[nt][1]) * fa : -CUDART_INF_F;
+      sv[2] = vb ? ((acc[nt][2] + acc2[nt][2]) - qbias[nt][0]) * fb : -CUDART_INF_F;
+      sv[3] = vb ? ((acc[nt][3] + acc2[nt][3]) - qbias[nt][1]) * fb : -CUDART_INF_F;
       float pr[4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float mx = fmaxf(s[j], s[j + 2]);
+      for (int jj = 0; jj < 2; ++jj) {
+        float mx = fmaxf(sv[jj], sv[jj + 2]);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[nt][j], mx);
+        const float m_new = fmaxf(m_run[nt][jj], mx);
         const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-        const float alpha = exp2f(m_run[nt][j] - m_use);
-        pr[j] = exp2f(s[j] - m_use);
-        pr[j + 2] = exp2f(s[j + 2] - m_use);
-        l_run[nt][j] = l_run[nt][j] * alpha + pr[j] + pr[j + 2];
-        m_run[nt][j] = m_new;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          o[mt][nt][j] *= alpha;
-          o[mt][nt][j + 2] *= alpha;
-        }
+        const float a = fast_exp2(m_run[nt][jj] - m_use);
+        pr[jj] = fast_exp2(sv[jj] - m_use);
+        pr[jj + 2] = fast_exp2(sv[jj + 2] - m_use);
+        l_run[nt][jj] = l_run[nt][jj] * a + pr[jj] + pr[jj + 2];
+        m_run[nt][jj] = m_new;
+        alpha[nt][jj] = a;
+        rescale |= (a != 1.f);
       }
-      // P (token-major fragment) -> P^T B operand; hi/lo split keeps precision
       const float q0 = pr[0] * pva, q1 = pr[1] * pva, q2 = pr[2] * pvb, q3 = pr[3] * pvb;
+      if constexpr (I8) {
+        p_run[nt][0] = p_run[nt][0] * alpha[nt][0] + (q0 + q2);
+        p_run[nt][1] = p_run[nt][1] * alpha[nt][1] + (q1 + q3);
+      }
       uint32_t h01, h23, l01, l23;
       if constexpr (!I8) {
         h01 = pack_bf16(q0, q1);
@@ -433,33 +611,41 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       bl[nt][0] = movmatrix_trans(l01);
       bl[nt][1] = movmatrix_trans(l23);
     }
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          o[mt][nt][0] *= alpha[nt][0];
+          o[mt][nt][2] *= alpha[nt][0];
+          o[mt][nt][1] *= alpha[nt][1];
+          o[mt][nt][3] *= alpha[nt][1];
+        }
+    }
 
     // ---- O^T[d][head] += V^T * P^T
     if constexpr (!I8) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4_trans(vS + swz<CH>(lm_row_v, 2 * mt + lm_ch_v) * 16, a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          mma_bf16(o[mt][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-          mma_bf16(o[mt][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bh[nt][0], bh[nt][1]);
+          mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bl[nt][0], bl[nt][1]);
         }
       }
     } else {
 #pragma unroll
       for (int mp = 0; mp < MT / 2; ++mp) {
-        uint32_t r0, r1, r2, r3;  // (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1)
-        ldmatrix_x4_trans(vS + swz<CH>(lm_row_a, 2 * mp + lm_ch_a) * 16, r0, r1, r2, r3);
-        const uint32_t top[2] = {r0 ^ 0x80808080u, r2 ^ 0x80808080u};
-        const uint32_t bot[2] = {r1 ^ 0x80808080u, r3 ^ 0x80808080u};
+        // vf[mp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1), transposed
+        const uint32_t top[2] = {vf[mp][0] ^ 0x80808080u, vf[mp][2] ^ 0x80808080u};
+        const uint32_t bot[2] = {vf[mp][1] ^ 0x80808080u, vf[mp][3] ^ 0x80808080u};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           // rows m <-> d: m = g -> 16c + 2g, m = g + 8 -> 16c + 2g + 1
-          const uint32_t a0 = i8pair_to_f16x2<0x4240>(top[h]);
-          const uint32_t a1 = i8pair_to_f16x2<0x4341>(top[h]);
-          const uint32_t a2 = i8pair_to_f16x2<0x4240>(bot[h]);
-          const uint32_t a3 = i8pair_to_f16x2<0x4341>(bot[h]);
+          const uint32_t a0 = i8pair_to_f16x2_biased<0x4240>(top[h]);
+          const uint32_t a1 = i8pair_to_f16x2_biased<0x4341>(top[h]);
+          const uint32_t a2 = i8pair_to_f16x2_biased<0x4240>(bot[h]);
+          const uint32_t a3 = i8pair_to_f16x2_biased<0x4341>(bot[h]);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
@@ -468,11 +654,28 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         }
       }
     }
-    __syncwarp();
   }
   cp_async_wait<0>();
 
-  // ---- per-warp final state -> smem (ring is reused: wait for every warp)
+  if constexpr (I8) {
+    // O carries 1152 * sum_t P[t][h] from the biased V codes: remove it.
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float ps = p_run[nt][j];
+        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          o[mt][nt][j] -= 1152.f * ps;
+          o[mt][nt][j + 2] -= 1152.f * ps;
+        }
+      }
+  }
+
+  // ---- per-warp final state -> smem (the ring is reused: wait for every warp)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -716,9 +919,9 @@ __global__ void __launch_bounds__(HD) merge_kernel(const DecodeParams p) {
 namespace {
 
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel) to
-// the largest size any launch can ask for; later launches skip the runtime
-// call.  The flag array is per kernel (the kernel is the template argument).
-// Racing first calls from several host threads both set the same value.
+// the device's opt-in maximum; later launches skip the runtime call.  The
+// cached limit is per kernel (the kernel is the template argument).  Racing
+// first calls from several host threads set the same value.
 constexpr int kMaxDevices = 64;
 
 template <auto Kernel>
@@ -743,19 +946,10 @@ cudaError_t prepare(int smem) {
 }
 
 template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
-int mma_smem(const DecodeParams& p) {
-  constexpr int ELEM = I8 ? 1 : 2;
-  constexpr int STAGE_B = 2 * 16 * HD * ELEM + (I8 ? 128 : 0);
-  constexpr int RING = NWARPS * NSTAGES * STAGE_B;
-  constexpr int GP = NT * 8;
-  constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
-  return p.phys_bytes + (RING > COMB ? RING : COMB);
-}
-
-template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = MmaCfg<HD, I8, NT, NWARPS, NSTAGES>;
+  const int smem = p.phys_bytes + Cfg::BODY;
   constexpr auto k = decode_mma_kernel<HD, I8, NT, NWARPS, NSTAGES>;
-  const int smem = mma_smem<HD, I8, NT, NWARPS, NSTAGES>(p);
   cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
@@ -778,22 +972,45 @@ cudaError_t launch_simt(const DecodeParams& p, dim3 grid, cudaStream_t st) {
 
 }  // namespace
 
-// Tile-engine configuration per cache type (warps per CTA, ring depth).
-constexpr int kBf16Warps = 4, kBf16Stages = 3;
-constexpr int kI8Warps = 4, kI8Stages = 4;
 constexpr int kF32Warps = 4, kF32Stages = 2;
+constexpr int kMW = PKV_MMA_WARPS;
+
+namespace {
+
+template <auto Kernel>
+int occupancy(int threads, int smem) {
+  static std::atomic<int> cached[kMaxDevices];  // resident CTAs per SM, 0 = not yet
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  int n = cached[dev].load(std::memory_order_acquire);
+  if (n > 0) return n;
+  if (prepare<Kernel>(smem) != cudaSuccess) return 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  cached[dev].store(n, std::memory_order_release);
+  return n;
+}
+
+constexpr int kTypicalPhysBytes = 1024;  // block-table slice of a typical split
+
+template <int HD, bool I8>
+int mma_occupancy() {
+  using Cfg = MmaCfg<HD, I8, 1, kMW, I8 ? PKV_I8_STAGES : PKV_BF16_STAGES>;
+  return occupancy<decode_mma_kernel<HD, I8, 1, kMW, I8 ? PKV_I8_STAGES : PKV_BF16_STAGES>>(
+      kMW * kWarp, kTypicalPhysBytes + Cfg::BODY);
+}
+
+}  // namespace
 
 int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim) {
-  // resident CTAs per SM implied by the shared-memory ring (228 KB per SM)
-  int ring;
-  if (cache_dt == PKV_BF16)
-    ring = kBf16Warps * kBf16Stages * 2 * 16 * head_dim * 2;
-  else if (cache_dt == PKV_I8)
-    ring = kI8Warps * kI8Stages * (2 * 16 * head_dim + 128);
-  else
-    ring = kF32Warps * kF32Stages * 2 * 16 * head_dim * 4 + 16 * head_dim * 4;
-  int n = (228 * 1024) / (ring + 4096);
-  return n < 1 ? 1 : (n > 8 ? 8 : n);
+  if (cache_dt == PKV_BF16) return head_dim == 128 ? mma_occupancy<128, false>()
+                                                   : mma_occupancy<64, false>();
+  if (cache_dt == PKV_I8) return head_dim == 128 ? mma_occupancy<128, true>()
+                                                 : mma_occupancy<64, true>();
+  const int smem = kF32Warps * kF32Stages * 2 * 16 * head_dim * 4 + 16 * head_dim * 4 + 1024;
+  const int n = (228 * 1024) / (smem + 1024);
+  return n < 1 ? 1 : n;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
@@ -802,17 +1019,17 @@ cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_di
   const bool two = p.group > 8;
   if (cache_dt == PKV_BF16) {
     if (head_dim == 128)
-      return two ? launch_mma<128, false, 2, kBf16Warps, kBf16Stages>(p, grid, st)
-                 : launch_mma<128, false, 1, kBf16Warps, kBf16Stages>(p, grid, st);
-    return two ? launch_mma<64, false, 2, kBf16Warps, kBf16Stages>(p, grid, st)
-               : launch_mma<64, false, 1, kBf16Warps, kBf16Stages>(p, grid, st);
+      return two ? launch_mma<128, false, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
+                 : launch_mma<128, false, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
+    return two ? launch_mma<64, false, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
+               : launch_mma<64, false, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
   }
   if (cache_dt == PKV_I8) {
     if (head_dim == 128)
-      return two ? launch_mma<128, true, 2, kI8Warps, kI8Stages>(p, grid, st)
-                 : launch_mma<128, true, 1, kI8Warps, kI8Stages>(p, grid, st);
-    return two ? launch_mma<64, true, 2, kI8Warps, kI8Stages>(p, grid, st)
-               : launch_mma<64, true, 1, kI8Warps, kI8Stages>(p, grid, st);
+      return two ? launch_mma<128, true, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+                 : launch_mma<128, true, 1, kMW, PKV_I8_STAGES>(p, grid, st);
+    return two ? launch_mma<64, true, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+               : launch_mma<64, true, 1, kMW, PKV_I8_STAGES>(p, grid, st);
   }
   if (head_dim == 128) return launch_simt<128, kF32Warps, kF32Stages>(p, grid, st);
   return launch_simt<64, kF32Warps, kF32Stages>(p, grid, st);
