@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-copy-probe", action="store_true")
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared-prefix workload: read the shared blocks once per KV head")
     return ap.parse_args()
 
 
@@ -254,6 +256,7 @@ def config_dict(wl, args, splits):
         "num_q_heads": wl.num_q_heads, "num_kv_heads": wl.num_kv_heads,
         "head_dim": wl.head_dim, "block_size": wl.block_size, "cache_dtype": wl.cache_dtype,
         "num_blocks": wl.num_blocks, "num_splits": splits,
+        "shared_prefix_pass": bool(getattr(args, "cascade", False)),
         "step": "kv_cache_append (1 new token per sequence) + paged_attention_decode",
         "kv_bytes_per_step": wl.kv_bytes(),
         "l2": ("inputs larger than L2 (KV %d MB > 126 MB L2), no flush"
@@ -314,20 +317,40 @@ def main():
     bt, cl = wl.block_tables.to(dev), wl.context_lens.to(dev)
     max_ctx = wl.max_context_len
     cache_tdt = tdt
-    splits = args.num_splits or pkv.decode_num_splits(wl.num_seqs, wl.num_kv_heads, wl.head_dim,
-                                                       max_ctx, cache_tdt)
-    ws_bytes = pkv.workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                                  max_ctx, cache_tdt, splits)
+    prefix_len = int(wl.meta.get("shared_prefix", 0)) if args.cascade else 0
+    if args.cascade and prefix_len == 0:
+        raise SystemExit("--cascade needs a workload with a shared prefix")
+    if prefix_len:
+        suffix_max = max(max_ctx - prefix_len, 0)
+        splits = args.num_splits or pkv.decode_num_splits(wl.num_seqs, wl.num_kv_heads,
+                                                           wl.head_dim, suffix_max, cache_tdt)
+        ws_bytes = pkv.shared_prefix_workspace_size(wl.num_seqs, wl.num_q_heads,
+                                                    wl.num_kv_heads, wl.head_dim, max_ctx,
+                                                    prefix_len, cache_tdt, splits)
+    else:
+        splits = args.num_splits or pkv.decode_num_splits(wl.num_seqs, wl.num_kv_heads,
+                                                           wl.head_dim, max_ctx, cache_tdt)
+        ws_bytes = pkv.workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                                      max_ctx, cache_tdt, splits)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     out = torch.empty_like(q)
+
+    def attend(qq, btt, cll):
+        if prefix_len:
+            pkv.paged_attention_decode_shared_prefix(
+                qq, k_cache, v_cache, btt, cll, prefix_len, softmax_scale=wl.softmax_scale,
+                max_context_len=max_ctx, out=out, workspace=ws, num_splits=splits, err_flag=err)
+        else:
+            pkv.paged_attention_decode(qq, k_cache, v_cache, btt, cll,
+                                       softmax_scale=wl.softmax_scale, k_scale=k_scale,
+                                       v_scale=v_scale, max_context_len=max_ctx, out=out,
+                                       workspace=ws, num_splits=splits, err_flag=err)
 
     def step(ev_pair=None):
         pkv.kv_cache_append(nk, nv, ns, k_cache, v_cache, k_scale, v_scale, err_flag=err)
         if ev_pair is not None:
             ev_pair[0].record()
-        pkv.paged_attention_decode(q, k_cache, v_cache, bt, cl, softmax_scale=wl.softmax_scale,
-                                   k_scale=k_scale, v_scale=v_scale, max_context_len=max_ctx,
-                                   out=out, workspace=ws, num_splits=splits, err_flag=err)
+        attend(q, bt, cl)
         if ev_pair is not None:
             ev_pair[1].record()
 
@@ -417,10 +440,7 @@ def main():
             dbt.copy_(hbt, non_blocking=True)
             dcl.copy_(hcl, non_blocking=True)
             pkv.kv_cache_append(dk, dv, dsl, k_cache, v_cache, k_scale, v_scale, err_flag=err)
-            pkv.paged_attention_decode(dq, k_cache, v_cache, dbt, dcl,
-                                       softmax_scale=wl.softmax_scale, k_scale=k_scale,
-                                       v_scale=v_scale, max_context_len=max_ctx, out=out,
-                                       workspace=ws, num_splits=splits, err_flag=err)
+            attend(dq, dbt, dcl)
             hout.copy_(out, non_blocking=True)
 
         for _ in range(W):
@@ -450,7 +470,7 @@ def main():
     if rank == 0:
         ms_per_step = max_ms / K
         layers = LAYERS.get(wl.name, 1)
-        launches_per_step = 2 + (1 if splits > 1 else 0)
+        launches_per_step = (4 if prefix_len else 2 + (1 if splits > 1 else 0))
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5),
@@ -465,7 +485,9 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic,
-                         "kernel": "pkv_paged_attention_decode (decode + split merge)",
+                         "kernel": ("pkv_paged_attention_decode_shared_prefix (prefix pass + "
+                                    "suffix decode + merge; logical KV bytes)" if prefix_len else
+                                    "pkv_paged_attention_decode (decode + split merge)"),
                          "peak_source": f"{peak_kind} (hbm_gbs)",
                          "decode_ms_mean": round(decode_ms, 5),
                          "decode_ms_min": round(min(call_ms), 5)},

@@ -147,6 +147,38 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
                                int num_splits, int* err_flag, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_decode_shared_prefix - pkv_paged_attention_decode for a
+ * batch whose sequences all begin with the same `prefix_len` tokens stored in
+ * the same physical blocks (prefix caching: "生产级 LLM 推理的 KV 缓存优化"
+ * (GPUYard), serving flags, --enable-prefix-caching; shared blocks with a
+ * ref_count: [mlqm] §2).  The result is the same attention as
+ * pkv_paged_attention_decode; only the order of the work differs: the shared
+ * blocks are read once per KV head for all sequences (a dense q-rows x tokens
+ * contraction), each sequence's remaining tokens are attended separately, and
+ * the partials are merged through their log-sum-exp.
+ *
+ * Arguments as for pkv_paged_attention_decode, plus:
+ *   prefix_len    host int, a multiple of block_size, <= max_blocks_per_seq *
+ *                 block_size.  The prefix blocks are read from sequence 0's
+ *                 block table; every sequence's table must hold the same
+ *                 entries there (sequences shorter than prefix_len attend to
+ *                 their first context_lens tokens only).  0 = plain decode.
+ *   workspace     >= pkv_shared_prefix_workspace_size(...) bytes (always needed
+ *                 when prefix_len > 0).
+ * Supported: cache_dt == PKV_BF16 (others: PKV_ERR_UNSUPPORTED), q_dt == PKV_BF16.
+ */
+size_t pkv_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                        int head_dim, int max_context_len, int prefix_len,
+                                        pkv_dtype cache_dt, int num_splits);
+int pkv_paged_attention_decode_shared_prefix(
+    void* out, const void* q, pkv_dtype q_dt, const void* k_cache, const void* v_cache,
+    pkv_dtype cache_dt, const float* k_scale, const float* v_scale, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+    float softmax_scale, int prefix_len, void* workspace, size_t workspace_bytes, int num_splits,
+    int* err_flag, pkv_stream_t stream);
+
+/*
  * pkv_copy - device-to-device copy of `bytes` bytes (a multiple of 16) with a
  * streaming kernel; used to measure the attainable HBM bandwidth in the same
  * process as the attention kernels.  Not part of the attention path.

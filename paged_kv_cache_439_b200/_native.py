@@ -33,6 +33,10 @@ SIGNATURES = {
     "pkv_paged_attention_decode_noalloc": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i,
                                                 _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                                                 _vp]),
+    "pkv_shared_prefix_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "pkv_paged_attention_decode_shared_prefix": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp,
+                                                      _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                                                      _i, _vp, _sz, _i, _vp, _vp]),
     "pkv_copy": (_i, [_vp, _vp, _sz, _vp]),
     "pkv_strerror": (ctypes.c_char_p, [_i]),
     "pkv_version": (_i, []),

@@ -150,6 +150,52 @@ def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor,
     return out
 
 
+def shared_prefix_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                 head_dim: int, max_context_len: int, prefix_len: int,
+                                 cache_dtype: torch.dtype, num_splits: int = 0) -> int:
+    return int(N.lib().pkv_shared_prefix_workspace_size(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_len,
+        _DT[cache_dtype], num_splits))
+
+
+def paged_attention_decode_shared_prefix(q: torch.Tensor, k_cache: torch.Tensor,
+                                         v_cache: torch.Tensor, block_tables: torch.Tensor,
+                                         context_lens: torch.Tensor, prefix_len: int,
+                                         softmax_scale: Optional[float] = None,
+                                         max_context_len: Optional[int] = None,
+                                         out: Optional[torch.Tensor] = None,
+                                         workspace: Optional[torch.Tensor] = None,
+                                         num_splits: int = 0,
+                                         err_flag: Optional[torch.Tensor] = None,
+                                         stream=None) -> torch.Tensor:
+    """Decode attention for a batch whose sequences share their first
+    ``prefix_len`` tokens (same physical blocks, taken from sequence 0's table).
+    Same result as paged_attention_decode; the shared blocks are read once per
+    KV head for all sequences."""
+    B, nq, d = q.shape
+    nb, bs, nkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        need = shared_prefix_workspace_size(B, nq, nkv, d, max_context_len, prefix_len,
+                                            k_cache.dtype, num_splits)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    rc = N.lib().pkv_paged_attention_decode_shared_prefix(
+        _ptr(out), _ptr(q), _dt(q), _ptr(k_cache), _ptr(v_cache), _dt(k_cache), None, None,
+        _ptr(block_tables), maxb, _ptr(context_lens), max_context_len, B, nq, nkv, d, bs, nb,
+        float(softmax_scale), prefix_len, _ptr(workspace), workspace.numel(), num_splits,
+        _ptr(err_flag), _stream(stream))
+    N.check(rc, "pkv_paged_attention_decode_shared_prefix")
+    return out
+
+
 def copy(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
     """Streaming device copy (HBM bandwidth probe)."""
     nbytes = src.numel() * src.element_size()

@@ -91,6 +91,37 @@ size_t ws_bytes(int num_seqs, int num_q_heads, int head_dim, int splits) {
 
 int map_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
+// Shared-prefix plan: prefix slices (about two CTAs per SM over KV heads and
+// row groups), then the suffix splits of the remaining context.
+struct PrefixPlan {
+  int ps, pchunk;      // prefix slices and their length
+  int splits, chunk;   // suffix splits
+  int slots;           // workspace partials per (sequence, q head)
+  size_t ws;           // workspace bytes
+};
+
+PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                       int max_ctx, int prefix_len, pkv_dtype cache_dt, int num_splits) {
+  PrefixPlan pl;
+  const long long rows = (long long)num_seqs * (num_q_heads / num_kv_heads);
+  const long long rg = (rows + pkv::prefix_rows_per_cta() - 1) / pkv::prefix_rows_per_cta();
+  const long long target = 2LL * sm_count();
+  long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
+  const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;
+  if (ps > max_ps) ps = max_ps;
+  if (ps < 1) ps = 1;
+  pl.pchunk = round_up((int)((prefix_len + ps - 1) / ps), pkv::kPrefixTokens);
+  pl.ps = (prefix_len + pl.pchunk - 1) / pl.pchunk;
+  const int suffix = max_ctx > prefix_len ? max_ctx - prefix_len : 0;
+  int req = num_splits;
+  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, suffix, cache_dt);
+  plan(suffix, req, &pl.splits, &pl.chunk);
+  pl.slots = pl.ps + pl.splits;
+  const size_t r = (size_t)num_seqs * num_q_heads * pl.slots;
+  pl.ws = align256(r * head_dim * sizeof(float)) + align256(r * sizeof(float));
+  return pl;
+}
+
 }  // namespace
 
 extern "C" {
@@ -227,6 +258,10 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
   p.max_context_len = max_context_len;
   p.chunk = chunk;
   p.num_splits = splits;
+  p.t_start = 0;
+  p.ws_slots = splits;
+  p.ws_base = 0;
+  p.direct = splits == 1;
   p.phys_bytes = round_up((chunk / block_size + 2) * 4, 128);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   p.q_f32 = q_dt == PKV_F32;
@@ -247,6 +282,111 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
     e = pkv::launch_merge(p, head_dim, st);
     if (e != cudaSuccess) return PKV_ERR_CUDA;
   }
+  return PKV_OK;
+}
+
+size_t pkv_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                        int head_dim, int max_context_len, int prefix_len,
+                                        pkv_dtype cache_dt, int num_splits) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0 ||
+      num_splits < 0 || prefix_len < 0 || num_q_heads % num_kv_heads != 0)
+    return 0;
+  if (prefix_len == 0)
+    return pkv_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                              cache_dt, num_splits);
+  return plan_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_len,
+                     cache_dt, num_splits)
+      .ws;
+}
+
+int pkv_paged_attention_decode_shared_prefix(
+    void* out, const void* q, pkv_dtype q_dt, const void* k_cache, const void* v_cache,
+    pkv_dtype cache_dt, const float* k_scale, const float* v_scale, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+    float softmax_scale, int prefix_len, void* workspace, size_t workspace_bytes, int num_splits,
+    int* err_flag, pkv_stream_t stream) {
+  if (prefix_len < 0) return PKV_ERR_ARG;
+  if (prefix_len == 0)
+    return pkv_paged_attention_decode(out, q, q_dt, k_cache, v_cache, cache_dt, k_scale, v_scale,
+                                      block_tables, max_blocks_per_seq, context_lens,
+                                      max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                                      head_dim, block_size, num_blocks, softmax_scale, workspace,
+                                      workspace_bytes, num_splits, err_flag, stream);
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || num_splits < 0)
+    return PKV_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PKV_ERR_ARG;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PKV_ERR_ARG;
+  if (!isfinite(softmax_scale)) return PKV_ERR_ARG;
+  const int group = num_q_heads / num_kv_heads;
+  if (group > 16) return PKV_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
+  if (!pow2_in(block_size, 8, 256)) return PKV_ERR_SHAPE;
+  if (cache_dt != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (q_dt != PKV_BF16) return PKV_ERR_DTYPE;
+  if (prefix_len % block_size != 0 || (long long)prefix_len > (long long)max_blocks_per_seq * block_size)
+    return PKV_ERR_ARG;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(err_flag, 4) ||
+      !aligned(workspace, 16))
+    return PKV_ERR_ALIGN;
+  if (num_seqs == 0) return PKV_OK;
+  if (num_seqs > 65535) return PKV_ERR_UNSUPPORTED;
+
+  const long long cap = (long long)max_blocks_per_seq * block_size;
+  const int max_ctx = (int)(max_context_len < cap ? max_context_len : cap);
+  const int suffix = max_ctx > prefix_len ? max_ctx - prefix_len : 0;
+  if (num_splits != 0 && num_splits < min_splits(suffix)) return PKV_ERR_UNSUPPORTED;
+  const PrefixPlan pl = plan_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, max_ctx,
+                                    prefix_len, cache_dt, num_splits);
+  if (pl.splits < min_splits(suffix)) return PKV_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < pl.ws) return PKV_ERR_WORKSPACE;
+
+  pkv::DecodeParams p;
+  p.out = out;
+  p.q = q;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.err_flag = err_flag;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_seqs = num_seqs;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.block_size = block_size;
+  p.log2_bs = log2i(block_size);
+  p.num_blocks = num_blocks;
+  p.max_context_len = max_context_len;
+  p.chunk = pl.chunk;
+  p.num_splits = pl.splits;
+  p.t_start = prefix_len;
+  p.ws_slots = pl.slots;
+  p.ws_base = pl.ps;
+  p.direct = 0;
+  p.phys_bytes = round_up((pl.chunk / block_size + 2) * 4, 128);
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.q_f32 = 0;
+  p.out_f32 = 0;
+  const size_t rows = (size_t)num_seqs * num_q_heads * pl.slots;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                      align256(rows * head_dim * sizeof(float)));
+  pkv::PrefixParams pp;
+  pp.prefix_len = prefix_len;
+  pp.pchunk = pl.pchunk;
+  pp.prefix_splits = pl.ps;
+  pp.rows = num_seqs * group;
+  pp.phys_bytes = round_up((pl.pchunk / block_size + 2) * 4, 128);
+
+  cudaStream_t st = (cudaStream_t)stream;
+  if (pkv::launch_prefix(p, pp, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
+  if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
+  if (pkv::launch_merge(p, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }
 

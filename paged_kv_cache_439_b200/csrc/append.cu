@@ -22,7 +22,11 @@ namespace {
 
 constexpr int kAppendThreads = 128;
 
-// One CTA per token: K and V rows of num_kv_heads * head_dim elements.
+// Grid (token, K|V, row piece): each CTA copies kAppendThreads * kVecs 16-byte
+// vectors of one token's row (all KV heads).  Every thread issues all of its
+// loads before any store, so a launch costs one memory round trip.
+constexpr int kVecs = 4;
+
 __global__ void __launch_bounds__(kAppendThreads)
     append_copy_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                        const int64_t* __restrict__ slot_mapping, int row_vecs,
@@ -32,18 +36,22 @@ __global__ void __launch_bounds__(kAppendThreads)
   const long long slot = slot_mapping[t];
   if (slot < 0) return;
   if (slot >= num_slots) {
-    if (threadIdx.x == 0) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
+    if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
     return;
   }
-  const uint4* ks = k + (size_t)t * row_vecs;
-  const uint4* vs = v + (size_t)t * row_vecs;
-  uint4* kd = k_cache + (size_t)slot * row_vecs;
-  uint4* vd = v_cache + (size_t)slot * row_vecs;
-  for (int i = threadIdx.x; i < row_vecs; i += kAppendThreads) {
-    const uint4 a = __ldg(ks + i);
-    const uint4 b = __ldg(vs + i);
-    kd[i] = a;
-    vd[i] = b;
+  const uint4* src = (blockIdx.y ? v : k) + (size_t)t * row_vecs;
+  uint4* dst = (blockIdx.y ? v_cache : k_cache) + (size_t)slot * row_vecs;
+  const int first = blockIdx.z * (kAppendThreads * kVecs) + threadIdx.x;
+  uint4 buf[kVecs];
+#pragma unroll
+  for (int i = 0; i < kVecs; ++i) {
+    const int idx = first + i * kAppendThreads;
+    if (idx < row_vecs) buf[i] = __ldg(src + idx);
+  }
+#pragma unroll
+  for (int i = 0; i < kVecs; ++i) {
+    const int idx = first + i * kAppendThreads;
+    if (idx < row_vecs) dst[idx] = buf[i];
   }
 }
 
@@ -154,7 +162,8 @@ cudaError_t launch_append(const void* k, const void* v, const int64_t* slot_mapp
   }
   const int elem = (in_dt == PKV_F32) ? 4 : 2;
   const int row_vecs = num_kv_heads * head_dim * elem / 16;
-  append_copy_kernel<<<num_tokens, kAppendThreads, 0, st>>>(
+  const dim3 grid(num_tokens, 2, (row_vecs + kAppendThreads * kVecs - 1) / (kAppendThreads * kVecs));
+  append_copy_kernel<<<grid, kAppendThreads, 0, st>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, row_vecs,
       static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), num_slots, err_flag);
   return cudaGetLastError();

@@ -148,4 +148,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Smem index of the 16-byte chunk `ch` of tile row `row` (rows of CH chunks).
+// XOR-swizzle so that the 8 rows an ldmatrix phase reads hit 8 distinct bank
+// groups.
+template <int CH>
+__device__ __forceinline__ int swz(int row, int ch) {
+  if constexpr (CH >= 8) {
+    return row * CH + (ch ^ (row & 7));
+  } else {
+    static_assert(CH == 4, "rows of 4 or a multiple of 8 chunks");
+    return row * CH + (ch ^ ((row >> 1) & 3));
+  }
+}
+
 }  // namespace pkv

@@ -29,19 +29,6 @@
 
 namespace pkv {
 
-// Smem index of the 16-byte chunk `ch` of tile row `row` (rows of CH chunks).
-// XOR-swizzle so that the 8 rows an ldmatrix phase reads hit 8 distinct bank
-// groups.
-template <int CH>
-__device__ __forceinline__ int swz(int row, int ch) {
-  if constexpr (CH >= 8) {
-    return row * CH + (ch ^ (row & 7));
-  } else {
-    static_assert(CH == 4, "rows of 4 or a multiple of 8 chunks");
-    return row * CH + (ch ^ ((row >> 1) & 3));
-  }
-}
-
 struct CtaSetup {
   int seq, kvh, split;
   int t_begin, t_end;  // token range of this CTA
@@ -57,7 +44,7 @@ __device__ __forceinline__ int effective_ctx(const DecodeParams& p, int seq, boo
     ctx = 0;
   }
   const long long cap_tab = (long long)p.max_blocks_per_seq * p.block_size;
-  const long long cap_split = (long long)p.num_splits * p.chunk;
+  const long long cap_split = (long long)p.t_start + (long long)p.num_splits * p.chunk;
   if (ctx > p.max_context_len || ctx > cap_tab) {
     if (report) set_flag(p.err_flag, PKV_FLAG_CTX_RANGE);
   }
@@ -75,7 +62,7 @@ __device__ __forceinline__ CtaSetup cta_setup(const DecodeParams& p, int* s_phys
   c.split = blockIdx.z;
   const bool report = (c.kvh == 0 && c.split == 0 && threadIdx.x == 0);
   const int ctx = effective_ctx(p, c.seq, report);
-  c.t_begin = c.split * p.chunk;
+  c.t_begin = p.t_start + c.split * p.chunk;
   c.t_end = min(ctx, c.t_begin + p.chunk);
   c.active = c.t_begin < c.t_end;
   c.blk0 = c.t_begin >> p.log2_bs;
@@ -172,9 +159,9 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& p, const C
       L += wt * s_l[w * GP + h];
     }
     s_L[h] = L;
-    if (p.num_splits > 1 && threadIdx.x < G) {
-      const size_t r = ((size_t)c.seq * p.num_q_heads + (size_t)c.kvh * G + h) * p.num_splits +
-                       c.split;
+    if (!p.direct && threadIdx.x < G) {
+      const size_t r = ((size_t)c.seq * p.num_q_heads + (size_t)c.kvh * G + h) * p.ws_slots +
+                       p.ws_base + c.split;
       p.ws_lse[r] = (L > 0.f) ? M + log2f(L) : -CUDART_INF_F;
     }
   }
@@ -187,7 +174,7 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& p, const C
     for (int w = 0; w < NWARPS; ++w) O += s_w[w * GP + h] * s_o[(w * GP + h) * HD + d];
     const float val = (L > 0.f) ? O / L : 0.f;
     const size_t qh = (size_t)c.kvh * G + h;
-    if (p.num_splits == 1) {
+    if (p.direct) {
       const size_t o = ((size_t)c.seq * p.num_q_heads + qh) * HD + d;
       if (p.out_f32)
         static_cast<float*>(p.out)[o] = val;
@@ -195,17 +182,17 @@ __device__ __forceinline__ void combine_and_store(const DecodeParams& p, const C
         static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(val);
     } else {
       const size_t o =
-          (((size_t)c.seq * p.num_q_heads + qh) * p.num_splits + c.split) * HD + d;
+          (((size_t)c.seq * p.num_q_heads + qh) * p.ws_slots + p.ws_base + c.split) * HD + d;
       p.ws_o[o] = val;
     }
   }
 }
 
 // Writes zeros for a sequence with nothing to attend (only the split-0 CTA of
-// a single-split launch; the merge kernel covers the multi-split case).
+// a direct launch; the merge kernel covers the other cases).
 template <int HD>
 __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup& c) {
-  if (p.num_splits != 1 || c.split != 0) return;
+  if (!p.direct || c.split != 0) return;
   const int G = p.group;
   for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
     const int h = idx / HD, d = idx % HD;
@@ -884,20 +871,23 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 }
 
 // ---------------------------------------------------------------------------
-// Split merge: out = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k} over the splits that
-// hold tokens.  One CTA per (q head, sequence), one thread per head_dim column.
+// Split merge: out = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k} over the partials
+// of one (sequence, q head): the shared-prefix slots [0, ws_base) and the
+// splits that hold tokens.  One CTA per (q head, sequence), one thread per
+// head_dim column.
 template <int HD>
 __global__ void __launch_bounds__(HD) merge_kernel(const DecodeParams p) {
   const int qh = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
   const int ctx = effective_ctx(p, seq, false);
-  const int n_valid = (ctx + p.chunk - 1) / p.chunk;
-  const size_t r = ((size_t)seq * p.num_q_heads + qh) * p.num_splits;
+  const int rest = ctx > p.t_start ? ctx - p.t_start : 0;
+  const int n = p.ws_base + (rest + p.chunk - 1) / p.chunk;
+  const size_t r = ((size_t)seq * p.num_q_heads + qh) * p.ws_slots;
   float M = -CUDART_INF_F;
-  for (int k = 0; k < n_valid; ++k) M = fmaxf(M, p.ws_lse[r + k]);
+  for (int k = 0; k < n; ++k) M = fmaxf(M, p.ws_lse[r + k]);
   float val = 0.f;
   if (M != -CUDART_INF_F) {
     float L = 0.f, O = 0.f;
-    for (int k = 0; k < n_valid; ++k) {
+    for (int k = 0; k < n; ++k) {
       const float lse = p.ws_lse[r + k];
       if (lse == -CUDART_INF_F) continue;
       const float w = exp2f(lse - M);

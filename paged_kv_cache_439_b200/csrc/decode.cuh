@@ -26,14 +26,32 @@ struct DecodeParams {
   int max_context_len;
   int chunk;       // tokens per split (multiple of 16)
   int num_splits;
+  int t_start;     // first token the split kernels cover (0, or a shared prefix length)
+  int ws_slots;    // partial results per (sequence, q head) in the workspace
+  int ws_base;     // workspace slot of split 0 (lower slots: shared-prefix partials)
+  int direct;      // 1: a single split writes `out` itself (no merge kernel)
   int phys_bytes;  // shared-memory bytes reserved for the block-table slice
   float scale_log2;  // softmax_scale * log2(e)
   int q_f32;
   int out_f32;
 };
 
+// Shared-prefix pass (prefix.cu): slices of the common prefix, all rows at once.
+struct PrefixParams {
+  int prefix_len;     // tokens at the start of every sequence held in shared blocks
+  int pchunk;         // prefix tokens per slice (a multiple of kPrefixTokens)
+  int prefix_splits;  // slices; slice i writes workspace slot i
+  int rows;           // q rows per KV head: num_seqs * group
+  int phys_bytes;     // shared-memory bytes for one slice's block-table entries
+};
+constexpr int kPrefixWarps = 8;    // 16 q rows per warp
+constexpr int kPrefixTokens = 64;  // tokens per shared-memory stage
+
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
                           cudaStream_t st);
+cudaError_t launch_prefix(const DecodeParams& p, const PrefixParams& pp, int head_dim,
+                          cudaStream_t st);
+int prefix_rows_per_cta();
 cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st);
 int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim);
 

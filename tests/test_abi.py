@@ -49,7 +49,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_strerror_and_version(lib):
     assert lib.pkv_strerror(0) == b"ok"
-    for s in range(-7, 0):
+    for s in range(-8, 0):
         assert lib.pkv_strerror(s) and lib.pkv_strerror(s) != b"unknown pkv status"
     assert lib.pkv_version() >> 16 == 1
 
@@ -104,6 +104,28 @@ def test_append_argument_errors(lib):
     assert call(cdt=2) == -1                  # int8 cache without scales
     assert call(k=FAKE + 4) == -7
     assert call(T=0) == 0                     # empty append is a no-op
+
+
+def test_shared_prefix_argument_errors(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, q_dt=1, k=FAKE, v=FAKE, cdt=1, bt=FAKE, maxb=8, cl=FAKE,
+                 maxctx=128, B=2, nq=8, nkv=2, d=128, bs=16, nb=20, scale=0.1, prefix=32,
+                 ws=None, wsb=0, splits=0, err=None)
+        a.update(kw)
+        return lib.pkv_paged_attention_decode_shared_prefix(
+            a["out"], a["q"], a["q_dt"], a["k"], a["v"], a["cdt"], None, None, a["bt"],
+            a["maxb"], a["cl"], a["maxctx"], a["B"], a["nq"], a["nkv"], a["d"], a["bs"], a["nb"],
+            a["scale"], a["prefix"], a["ws"], a["wsb"], a["splits"], a["err"], None)
+    assert call(prefix=-16) == -1
+    assert call(prefix=24) == -1                 # not a multiple of block_size
+    assert call(prefix=16 * 9) == -1             # beyond the block-table capacity
+    assert call(cdt=2) == -4                     # int8 cache: not supported by this call
+    assert call(q_dt=0) == -2
+    assert call(nq=6, nkv=4) == -1
+    assert call() == -5                          # the prefix pass always needs a workspace
+    need = lib.pkv_shared_prefix_workspace_size(2, 8, 2, 128, 128, 32, 1, 0)
+    assert need > 0
+    assert call(B=0, ws=FAKE, wsb=need) == 0
 
 
 def test_workspace_sizes(lib):

@@ -1,0 +1,91 @@
+"""Shared-prefix (cascade) decode against the oracle and the plain decode.
+
+Sequences of a batch share their first ``prefix_len`` tokens through the same
+physical blocks (prefix caching).  The cascade call must give the attention
+of the definition (checked against the oracle), whatever the group size,
+head_dim, block size, row count or prefix/suffix split."""
+import numpy as np
+import pytest
+import torch
+
+import paged_kv_cache_439_b200 as pkv
+from paged_kv_cache_439_b200.workloads import make_custom, make_workload
+
+from pkv_testlib import GpuCache, OracleCache, assert_close, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def _cascade(g, wl, prefix_len, context_lens=None, **kw):
+    dev = g.device
+    cl = (wl.context_lens if context_lens is None else context_lens).to(dev)
+    return pkv.paged_attention_decode_shared_prefix(
+        wl.q.to(dev), g.k, g.v, wl.block_tables.to(dev), cl, prefix_len,
+        softmax_scale=wl.softmax_scale, max_context_len=int(cl.max()), err_flag=g.err, **kw)
+
+
+@pytest.mark.parametrize("group,d,bs", [(4, 128, 16), (1, 128, 16), (8, 128, 16), (16, 64, 16),
+                                        (4, 64, 8), (8, 128, 256), (2, 128, 32)])
+def test_shared_prefix_matches_oracle(group, d, bs):
+    prefix = 256 if bs == 256 else 4 * bs * 8
+    lens = [prefix + x for x in (1, 17, 100, 5, 64, 300)]
+    wl = make_custom(f"sp-{group}-{d}-{bs}", lens, 2 * group, 2, d, bs, "bf16", seed=31,
+                     shared_prefix=prefix)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1, 3):
+        out = _cascade(g, wl, prefix, num_splits=splits)
+        assert_close(out, ref, tol_for(wl), f"{wl.name} splits={splits}")
+    assert g.flags() == 0
+    # and it agrees with the plain decode of the same cache
+    plain = g.decode()
+    np.testing.assert_allclose(_cascade(g, wl, prefix).float().cpu().numpy(),
+                               plain.float().cpu().numpy(), rtol=2e-2, atol=4e-3)
+
+
+def test_many_rows_span_several_row_groups():
+    # 40 sequences x group 8 = 320 q rows per KV head (several CTAs of rows)
+    lens = [128 + 1 + (7 * i) % 90 for i in range(40)]
+    wl = make_custom("sp-rows", lens, 16, 2, 128, 16, "bf16", seed=32, shared_prefix=128)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    assert_close(_cascade(g, wl, 128), ref, tol_for(wl), "rows")
+
+
+def test_sequences_shorter_than_the_prefix():
+    wl = make_custom("sp-short", [200, 150, 300], 8, 2, 128, 16, "bf16", seed=33, shared_prefix=128)
+    g = GpuCache(wl).fill()
+    cl = torch.tensor([200, 40, 0], dtype=torch.int32)   # 40 < prefix, 0 = empty
+    out = _cascade(g, wl, 128, context_lens=cl)
+    ref = OracleCache(wl).fill()
+    wl.context_lens = cl
+    r = ref.decode()
+    assert_close(out, r, tol_for(wl), "short")
+    assert (out[2] == 0).all()
+
+
+def test_prefix_only_and_bad_prefix_block():
+    wl = make_custom("sp-edge", [129, 130], 4, 1, 128, 16, "bf16", seed=34, shared_prefix=128)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    assert_close(_cascade(g, wl, 128), ref, tol_for(wl), "edge")
+    bt = wl.block_tables.clone()
+    bt[0, 2] = wl.num_blocks + 5                  # a bad entry inside the shared prefix
+    out = pkv.paged_attention_decode_shared_prefix(
+        wl.q.cuda(), g.k, g.v, bt.cuda(), wl.context_lens.cuda(), 128,
+        softmax_scale=wl.softmax_scale, max_context_len=130, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert g.flags() & 1
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("bs", [16, 256])
+def test_full_shared_prefix_workload(bs):
+    wl = make_workload("shared-prefix", block_size=bs)
+    g = GpuCache(wl).fill()
+    out = _cascade(g, wl, 4096)
+    torch.cuda.synchronize()
+    ref = OracleCache(wl).fill().decode()
+    r = assert_close(out, ref, tol_for(wl), f"shared-prefix bs={bs}")
+    assert g.flags() == 0
+    print(f"shared-prefix cascade bs={bs}: max_abs={r['max_abs']:.2e}")
