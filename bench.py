@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-copy-probe", action="store_true")
+    ap.add_argument("--kv-dtype", choices=["bf16", "i8", "fp8"], default=None,
+                    help="override the workload's KV-cache format")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix workload: read the shared blocks once per KV head")
     return ap.parse_args()
@@ -291,14 +293,17 @@ def main():
     from paged_kv_cache_439_b200 import dist as pdist
     from paged_kv_cache_439_b200.workloads import make_workload, workload_seed
 
+    extra = {"cache_dtype": args.kv_dtype} if args.kv_dtype else {}
     wl = make_workload(args.workload, block_size=args.block_size,
-                       data_seed=pdist.replica_seed(workload_seed(args.workload), rank))
-    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8}[wl.cache_dtype]
+                       data_seed=pdist.replica_seed(workload_seed(args.workload), rank), **extra)
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8,
+           "fp8": torch.float8_e4m3fn}[wl.cache_dtype]
     shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
-    k_cache = torch.zeros(shape, dtype=tdt, device=dev)
-    v_cache = torch.zeros(shape, dtype=tdt, device=dev)
+    k_cache = torch.zeros(shape, dtype=torch.uint8 if tdt == torch.float8_e4m3fn else tdt,
+                          device=dev).view(tdt)
+    v_cache = torch.zeros_like(k_cache)
     k_scale = v_scale = None
-    if wl.cache_dtype == "i8":
+    if wl.cache_dtype in ("i8", "fp8"):
         sshape = (wl.num_blocks, wl.num_kv_heads, wl.block_size)
         k_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
         v_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
@@ -475,7 +480,8 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": wl.cache_dtype if wl.cache_dtype != "i8" else "int8-kv/bf16-q",
+            "dtype": {"i8": "int8-kv/bf16-q", "fp8": "fp8e4m3-kv/bf16-q"}.get(wl.cache_dtype,
+                                                                           wl.cache_dtype),
             "data": "synthetic (seeded N(0,1) K/V/q shaped like the workload; no weights)",
             "config": config_dict(wl, args, splits),
             "pct_of_hbm_peak": round(100 * achieved / peak, 1),

@@ -12,7 +12,7 @@
  *          One physical block holds block_size token rows of all KV heads
  *          ([mlqm] §2, the Block class: k_data/v_data of block_size x hidden).
  *   scales k_scale, v_scale : fp32 [num_blocks][num_kv_heads][block_size]
- *          (INT8 caches only; one scale per token per head, [mlqm] §4).
+ *          (INT8 and FP8 caches only; one scale per token per head, [mlqm] §4).
  *   slot   physical_block * block_size + offset_in_block.
  *   table  block_tables     : int32 [num_seqs][max_blocks_per_seq]; entry j is
  *          the physical block of logical block j ([yunthe], PagedAttention
@@ -41,7 +41,9 @@ extern "C" {
 
 typedef struct CUstream_st* pkv_stream_t; /* identical to cudaStream_t */
 
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_I8 = 2 } pkv_dtype;
+/* PKV_FP8: E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * largest finite value 448) with one fp32 scale per token per head, like PKV_I8. */
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_I8 = 2, PKV_FP8 = 3 } pkv_dtype;
 
 typedef enum {
   PKV_OK = 0,
@@ -76,13 +78,18 @@ typedef enum {
  * (quantize_tensor): scale = 127 / max|x| over head_dim and code =
  * clamp(rint(x * scale), -128, 127), all in fp32, round-half-to-even, no fused
  * multiply-add; an all-zero row stores codes 0 and scale 1.  The scale goes to
- * k_scale/v_scale[block][head][row].
+ * k_scale/v_scale[block][head][row].  With cache_dt == PKV_FP8 (the pages'
+ * --kv-cache-dtype fp8: [gpuyard] serving flags, [yunthe] KV quantisation) the
+ * same per-row rule uses scale = 448 / max|x| and code = E4M3(x * scale),
+ * rounded to nearest even and saturated to +-448, in fp32.
  *
  *   k, v          device, [num_tokens][num_kv_heads][head_dim], dtype in_dt
  *                 (PKV_F32 or PKV_BF16), contiguous.  Read only.
  *   slot_mapping  device int64 [num_tokens].
- *   k_cache, v_cache  device, cache layout above, dtype cache_dt (== in_dt, or PKV_I8).
- *   k_scale, v_scale  device fp32 scale arrays; required iff cache_dt == PKV_I8.
+ *   k_cache, v_cache  device, cache layout above, dtype cache_dt (== in_dt, PKV_I8
+ *                 or PKV_FP8).
+ *   k_scale, v_scale  device fp32 scale arrays; required iff cache_dt is PKV_I8 or
+ *                 PKV_FP8.
  *   err_flag      device int or NULL (PKV_FLAG_BAD_SLOT).
  * Two tokens with the same slot race (last writer wins, unspecified).
  */
@@ -117,15 +124,15 @@ size_t pkv_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int h
  * h / (num_q_heads / num_kv_heads)).  For sequence s with c = context_lens[s]:
  *     out[s][h] = sum_t softmax_t(softmax_scale * <q[s][h], K_s[t]>) V_s[t],
  *     K_s[t] = k_cache[block_tables[s][t / block_size]][t % block_size][h / group]
- * over 0 <= t < c (c = 0 gives zeros).  INT8 caches are dequantised as
- * code / scale on load.  Long contexts are cut into num_splits splits whose
+ * over 0 <= t < c (c = 0 gives zeros).  INT8 and FP8 caches are dequantised as
+ * value(code) / scale on load.  Long contexts are cut into num_splits splits whose
  * partial results are merged exactly through their log-sum-exp.
  *
  *   out           device [num_seqs][num_q_heads][head_dim], dtype q_dt.  Written.
  *   q             device [num_seqs][num_q_heads][head_dim], dtype q_dt:
- *                 PKV_BF16 for BF16/I8 caches; PKV_F32 or PKV_BF16 for F32 caches.
- *   k_cache, v_cache, k_scale, v_scale  as above (scales only for PKV_I8; the
- *                 scale arrays must be 16-byte aligned here).
+ *                 PKV_BF16 for BF16/I8/FP8 caches; PKV_F32 or PKV_BF16 for F32 caches.
+ *   k_cache, v_cache, k_scale, v_scale  as above (scales only for PKV_I8 and
+ *                 PKV_FP8; the scale arrays must be 16-byte aligned here).
  *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past the
  *                 sequence's last block are never read.
  *   context_lens  device int32 [num_seqs].

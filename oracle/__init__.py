@@ -27,6 +27,11 @@ __all__ = [
     "paged_decode",
     "paged_decode_i8",
     "max_threads",
+    "e4m3_decode",
+    "e4m3_encode",
+    "quantize_row_fp8",
+    "append_fp8",
+    "paged_decode_fp8",
 ]
 
 _LIB = None
@@ -57,6 +62,16 @@ def _lib():
         lib.oracle_paged_decode_f32.argtypes = [_vp] * 5 + [_i32, _vp] + [_i32] * 6 + [_dbl, _i32]
         lib.oracle_paged_decode_i8.restype = _i32
         lib.oracle_paged_decode_i8.argtypes = [_vp] * 7 + [_i32, _vp] + [_i32] * 6 + [_dbl, _i32]
+        lib.oracle_e4m3_decode.restype = _dbl
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_quantize_row_fp8.restype = None
+        lib.oracle_quantize_row_fp8.argtypes = [_vp, _i32, _vp, _vp]
+        lib.oracle_append_fp8.restype = _i32
+        lib.oracle_append_fp8.argtypes = [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _i64, _i64]
+        lib.oracle_paged_decode_fp8.restype = _i32
+        lib.oracle_paged_decode_fp8.argtypes = [_vp] * 7 + [_i32, _vp] + [_i32] * 6 + [_dbl, _i32]
         lib.oracle_max_threads.restype = _i32
         lib.oracle_max_threads.argtypes = []
         _LIB = lib
@@ -179,4 +194,58 @@ def paged_decode_i8(q, k_codes, v_codes, k_scale, v_scale, block_tables, context
                                        bt.shape[1], clp, B, nq, nkv, d, bs, nb,
                                        float(softmax_scale), int(threads))
     _check(rc, "oracle_paged_decode_i8")
+    return out
+
+
+def e4m3_decode(code: int) -> float:
+    """Value of an E4M3 code (OCP FP8 definition)."""
+    return float(_lib().oracle_e4m3_decode(int(code) & 0xFF))
+
+
+def e4m3_encode(y: float) -> int:
+    """Nearest E4M3 code, ties to even, saturating at +-448."""
+    return int(_lib().oracle_e4m3_encode(float(y)))
+
+
+def quantize_row_fp8(x: np.ndarray):
+    """FP8 quantisation of one fp32 row.  Returns (codes uint8, scale)."""
+    xb, xp = _c(x, np.float32)
+    codes = np.zeros(xb.shape[0], dtype=np.uint8)
+    scale = np.zeros(1, dtype=np.float32)
+    _lib().oracle_quantize_row_fp8(xp, xb.shape[0], codes.ctypes.data_as(_vp),
+                                   scale.ctypes.data_as(_vp))
+    return codes, scale[0]
+
+
+def append_fp8(x: np.ndarray, slot_mapping: np.ndarray, codes: np.ndarray, scale: np.ndarray) -> None:
+    """FP8 quantising append, in place (layouts as append_int8, codes uint8)."""
+    xb, xp = _c(x, np.float32)
+    sm, sp = _c(slot_mapping, np.int64)
+    assert codes.dtype == np.uint8 and codes.flags.c_contiguous
+    assert scale.dtype == np.float32 and scale.flags.c_contiguous
+    nb, bs, nkv, d = codes.shape
+    assert scale.shape == (nb, nkv, bs) and xb.shape[1:] == (nkv, d)
+    rc = _lib().oracle_append_fp8(xp, sp, xb.shape[0], nkv, d, codes.ctypes.data_as(_vp),
+                                  scale.ctypes.data_as(_vp), nb, bs)
+    _check(rc, "oracle_append_fp8")
+
+
+def paged_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, block_tables, context_lens,
+                     softmax_scale, threads=0):
+    """fp64 paged decode attention over an FP8 cache (dequantised E4M3(code) / scale)."""
+    qb, qp = _c(q, np.float32)
+    kb, kp = _c(k_codes, np.uint8)
+    vb, vp = _c(v_codes, np.uint8)
+    ks, ksp = _c(k_scale, np.float32)
+    vs, vsp = _c(v_scale, np.float32)
+    bt, btp = _c(block_tables, np.int32)
+    cl, clp = _c(context_lens, np.int32)
+    B, nq, d = qb.shape
+    nb, bs, nkv, d2 = kb.shape
+    assert d == d2 and vb.shape == kb.shape and ks.shape == (nb, nkv, bs) == vs.shape
+    out = np.zeros((B, nq, d), dtype=np.float64)
+    rc = _lib().oracle_paged_decode_fp8(out.ctypes.data_as(_vp), qp, kp, vp, ksp, vsp, btp,
+                                        bt.shape[1], clp, B, nq, nkv, d, bs, nb,
+                                        float(softmax_scale), int(threads))
+    _check(rc, "oracle_paged_decode_fp8")
     return out

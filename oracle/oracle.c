@@ -26,6 +26,15 @@
  *    Dequantisation is code / scale (the page's dequant_matmul multiplies by
  *    the scales, which would be off by scale^2 given the definition above).
  *
+ *  - FP8 (E4M3) quantisation.  GPUYard, serving flags (--kv-cache-dtype fp8
+ *    halves the per-token cache) and yunthe.com, KV quantisation section
+ *    (FP8/INT8 KV).  The pages give no rule; the reading taken mirrors the
+ *    INT8 one: per token per head, scale = 448 / max|x| (448 = largest finite
+ *    E4M3 value), code = E4M3(x * scale) rounded to nearest-even and saturated
+ *    to +-448, all in fp32; dequantised value = E4M3 value / scale.  E4M3 is the
+ *    OCP 8-bit format: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no
+ *    infinities, S.1111.111 = NaN; subnormals 2^-6 * m/8.
+ *
  *  - Decode attention.  yunthe.com, PagedAttention section: the kernel looks
  *    up physical blocks through the block table, stitches the scattered K/V
  *    back together and runs standard attention.  mlqm.cn §3 (GQA example,
@@ -110,6 +119,86 @@ void oracle_quantize_row(const float* x, int n, int8_t* codes, float* scale_out)
   *scale_out = scale;
 }
 
+/* E4M3 value of an 8-bit code (NaN codes decode to NaN). */
+double oracle_e4m3_decode(uint8_t code) {
+  const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to y (ties to even mantissa), magnitudes above 448
+ * saturated to 448.  y must not be NaN. */
+uint8_t oracle_e4m3_encode(float y) {
+  const int sign = y < 0.0f || (y == 0.0f && signbit(y));
+  double a = fabs((double)y);
+  if (a >= 448.0) return (uint8_t)((sign << 7) | (15 << 3) | 6);
+  /* spacing of representable values around a: 2^(e-3) in binade [2^e, 2^(e+1)),
+   * e >= -6; below 2^-6 the subnormal spacing 2^-9 */
+  int ex;
+  frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1) */
+  int e = ex - 1;
+  if (a == 0.0 || e < -6) e = -6;
+  const double q = ldexp(1.0, e - 3);
+  const double mi = nearbyint(a / q); /* exact quotient, rounded half to even */
+  const double v = mi * q;            /* may reach 2^(e+1): still representable */
+  if (v >= 448.0) return (uint8_t)((sign << 7) | (15 << 3) | 6);
+  int code;
+  if (v < ldexp(1.0, -6)) {
+    code = (int)(v / ldexp(1.0, -9)); /* subnormal: m = v / 2^-9 */
+  } else {
+    int vx;
+    frexp(v, &vx);
+    const int ve = vx - 1;
+    const int m = (int)((v / ldexp(1.0, ve) - 1.0) * 8.0);
+    code = ((ve + 7) << 3) | m;
+  }
+  return (uint8_t)((sign << 7) | code);
+}
+
+/* FP8 quantisation of one fp32 row: scale = 448 / max|x|, codes E4M3(x*scale). */
+void oracle_quantize_row_fp8(const float* x, int n, uint8_t* codes, float* scale_out) {
+  float absmax = 0.0f;
+  for (int i = 0; i < n; ++i) {
+    float a = fabsf(x[i]);
+    if (a > absmax) absmax = a;
+  }
+  if (absmax == 0.0f) { /* same reading as INT8: codes 0, scale 1 */
+    for (int i = 0; i < n; ++i) codes[i] = 0;
+    *scale_out = 1.0f;
+    return;
+  }
+  float scale = 448.0f / absmax;
+  for (int i = 0; i < n; ++i) {
+    float y = x[i] * scale; /* one fp32 multiply, rounded */
+    codes[i] = oracle_e4m3_encode(y);
+  }
+  *scale_out = scale;
+}
+
+/* FP8 quantising append; layouts as oracle_append_int8. */
+int oracle_append_fp8(const float* x, const int64_t* slot_mapping, int64_t num_tokens,
+                      int num_kv_heads, int head_dim, uint8_t* codes, float* scale,
+                      int64_t num_blocks, int64_t block_size) {
+  if (!x || !slot_mapping || !codes || !scale || num_tokens < 0 || num_kv_heads <= 0 ||
+      head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+    return ORACLE_ERR_ARG;
+  for (int64_t t = 0; t < num_tokens; ++t) {
+    int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    int64_t block = slot / block_size;
+    int64_t offset = slot % block_size;
+    if (block >= num_blocks) return ORACLE_ERR_SLOT;
+    for (int h = 0; h < num_kv_heads; ++h) {
+      const float* row = x + (t * num_kv_heads + h) * (int64_t)head_dim;
+      uint8_t* dst = codes + ((block * block_size + offset) * num_kv_heads + h) * (int64_t)head_dim;
+      float* s = scale + (block * num_kv_heads + h) * block_size + offset;
+      oracle_quantize_row_fp8(row, head_dim, dst, s);
+    }
+  }
+  return ORACLE_OK;
+}
+
 /* Quantising append: x fp32 [num_tokens][num_kv_heads][head_dim].
  * codes: [num_blocks][block_size][num_kv_heads][head_dim] int8.
  * scale: [num_blocks][num_kv_heads][block_size] fp32 (one per token per head). */
@@ -152,18 +241,22 @@ static int gather_f32(double* dst, const float* cache, const int32_t* table_row,
   return ORACLE_OK;
 }
 
-/* Same walk for an INT8 cache, dequantising each value as code / scale. */
-static int gather_i8(double* dst, const int8_t* codes, const float* scale, const int32_t* table_row,
-                     int ctx, int num_kv_heads, int kvh, int head_dim, int block_size,
-                     int num_blocks) {
+/* Same walk for a quantised cache, dequantising each value as value(code) /
+ * scale, value(code) = the signed byte (INT8) or its E4M3 value (FP8). */
+static int gather_codes(double* dst, const uint8_t* codes, const float* scale,
+                        const int32_t* table_row, int ctx, int num_kv_heads, int kvh, int head_dim,
+                        int block_size, int num_blocks, int fp8) {
   const int64_t row = (int64_t)num_kv_heads * head_dim;
   for (int t = 0; t < ctx; ++t) {
     int32_t phys = table_row[t / block_size];
     if (phys < 0 || phys >= num_blocks) return ORACLE_ERR_BLOCK;
     int off = t % block_size;
-    const int8_t* src = codes + ((int64_t)phys * block_size + off) * row + (int64_t)kvh * head_dim;
+    const uint8_t* src = codes + ((int64_t)phys * block_size + off) * row + (int64_t)kvh * head_dim;
     double s = (double)scale[((int64_t)phys * num_kv_heads + kvh) * block_size + off];
-    for (int i = 0; i < head_dim; ++i) dst[(int64_t)t * head_dim + i] = (double)src[i] / s;
+    for (int i = 0; i < head_dim; ++i) {
+      double v = fp8 ? oracle_e4m3_decode(src[i]) : (double)(int8_t)src[i];
+      dst[(int64_t)t * head_dim + i] = v / s;
+    }
   }
   return ORACLE_OK;
 }
@@ -229,7 +322,7 @@ static int check_shapes(int num_seqs, int num_q_heads, int num_kv_heads, int hea
 /* One (sequence, kv head) problem: gather that head's K/V rows of the
  * sequence, then attend for each q head h with h / group == kvh. */
 static int decode_problem(double* out, const float* q, const float* k_cache, const float* v_cache,
-                          const int8_t* k_codes, const int8_t* v_codes, const float* k_scale,
+                          const uint8_t* k_codes, const uint8_t* v_codes, int fp8, const float* k_scale,
                           const float* v_scale, const int32_t* block_tables,
                           int max_blocks_per_seq, const int32_t* context_lens, int s, int kvh,
                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
@@ -243,11 +336,11 @@ static int decode_problem(double* out, const float* q, const float* k_cache, con
   const int32_t* trow = block_tables + (int64_t)s * max_blocks_per_seq;
   int e;
   if (k_codes) {
-    e = gather_i8(K, k_codes, k_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
-                  num_blocks);
+    e = gather_codes(K, k_codes, k_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
+                     num_blocks, fp8);
     if (!e)
-      e = gather_i8(V, v_codes, v_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
-                    num_blocks);
+      e = gather_codes(V, v_codes, v_scale, trow, ctx, num_kv_heads, kvh, head_dim, block_size,
+                       num_blocks, fp8);
   } else {
     e = gather_f32(K, k_cache, trow, ctx, num_kv_heads, kvh, head_dim, block_size, num_blocks);
     if (!e)
@@ -267,7 +360,7 @@ static int decode_problem(double* out, const float* q, const float* k_cache, con
 }
 
 static int decode_all(double* out, const float* q, const float* k_cache, const float* v_cache,
-                      const int8_t* k_codes, const int8_t* v_codes, const float* k_scale,
+                      const uint8_t* k_codes, const uint8_t* v_codes, int fp8, const float* k_scale,
                       const float* v_scale, const int32_t* block_tables, int max_blocks_per_seq,
                       const int32_t* context_lens, int num_seqs, int num_q_heads,
                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
@@ -282,7 +375,7 @@ static int decode_all(double* out, const float* q, const float* k_cache, const f
 #pragma omp parallel for schedule(dynamic, 1)
 #endif
   for (int64_t i = 0; i < problems; ++i) {
-    int e = decode_problem(out, q, k_cache, v_cache, k_codes, v_codes, k_scale, v_scale,
+    int e = decode_problem(out, q, k_cache, v_cache, k_codes, v_codes, fp8, k_scale, v_scale,
                            block_tables, max_blocks_per_seq, context_lens, (int)(i / num_kv_heads),
                            (int)(i % num_kv_heads), num_q_heads, num_kv_heads, head_dim,
                            block_size, num_blocks, softmax_scale);
@@ -306,7 +399,7 @@ int oracle_paged_decode_f32(double* out, const float* q, const float* k_cache,
                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                             int num_blocks, double softmax_scale, int num_threads) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return ORACLE_ERR_ARG;
-  return decode_all(out, q, k_cache, v_cache, NULL, NULL, NULL, NULL, block_tables,
+  return decode_all(out, q, k_cache, v_cache, NULL, NULL, 0, NULL, NULL, block_tables,
                     max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
                     head_dim, block_size, num_blocks, softmax_scale, num_threads);
 }
@@ -322,7 +415,23 @@ int oracle_paged_decode_i8(double* out, const float* q, const int8_t* k_codes,
                            double softmax_scale, int num_threads) {
   if (!out || !q || !k_codes || !v_codes || !k_scale || !v_scale || !block_tables || !context_lens)
     return ORACLE_ERR_ARG;
-  return decode_all(out, q, NULL, NULL, k_codes, v_codes, k_scale, v_scale, block_tables,
+  return decode_all(out, q, NULL, NULL, (const uint8_t*)k_codes, (const uint8_t*)v_codes, 0,
+                    k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                    num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, softmax_scale,
+                    num_threads);
+}
+
+/* Paged decode over an FP8 (E4M3) cache: codes and scales laid out as for
+ * INT8; values are dequantised as E4M3(code) / scale. */
+int oracle_paged_decode_fp8(double* out, const float* q, const uint8_t* k_codes,
+                            const uint8_t* v_codes, const float* k_scale, const float* v_scale,
+                            const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                            double softmax_scale, int num_threads) {
+  if (!out || !q || !k_codes || !v_codes || !k_scale || !v_scale || !block_tables || !context_lens)
+    return ORACLE_ERR_ARG;
+  return decode_all(out, q, NULL, NULL, k_codes, v_codes, 1, k_scale, v_scale, block_tables,
                     max_blocks_per_seq, context_lens, num_seqs, num_q_heads, num_kv_heads,
                     head_dim, block_size, num_blocks, softmax_scale, num_threads);
 }

@@ -11,7 +11,7 @@ import threading
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
 
-PKV_F32, PKV_BF16, PKV_I8 = 0, 1, 2
+PKV_F32, PKV_BF16, PKV_I8, PKV_FP8 = 0, 1, 2, 3
 
 PKV_FLAG_BAD_BLOCK = 1
 PKV_FLAG_BAD_SLOT = 2

@@ -12,7 +12,8 @@ import torch
 
 from . import _native as N
 
-_DT = {torch.float32: N.PKV_F32, torch.bfloat16: N.PKV_BF16, torch.int8: N.PKV_I8}
+_DT = {torch.float32: N.PKV_F32, torch.bfloat16: N.PKV_BF16, torch.int8: N.PKV_I8,
+       torch.float8_e4m3fn: N.PKV_FP8}
 
 
 def _dt(t: torch.Tensor) -> int:
@@ -44,8 +45,8 @@ def kv_cache_append(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor
                     err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     """Writes k, v [T, n_kv, d] into the paged caches at slot_mapping [T] (int64).
 
-    Caches are [num_blocks, block_size, n_kv, d]; for int8 caches the fp32
-    scales are [num_blocks, n_kv, block_size].
+    Caches are [num_blocks, block_size, n_kv, d]; for int8 and float8_e4m3fn
+    caches the fp32 scales are [num_blocks, n_kv, block_size].
     """
     T, nkv, d = k.shape
     nb, bs = k_cache.shape[0], k_cache.shape[1]

@@ -158,8 +158,9 @@ int pkv_kv_cache_append(const void* k, const void* v, const int64_t* slot_mappin
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
   if (!pow2_in(block_size, 8, 256)) return PKV_ERR_SHAPE;
   if (in_dt != PKV_F32 && in_dt != PKV_BF16) return PKV_ERR_DTYPE;
-  if (cache_dt != in_dt && cache_dt != PKV_I8) return PKV_ERR_DTYPE;
-  if (cache_dt == PKV_I8 && (!k_scale || !v_scale)) return PKV_ERR_ARG;
+  const bool coded = cache_dt == PKV_I8 || cache_dt == PKV_FP8;
+  if (cache_dt != in_dt && !coded) return PKV_ERR_DTYPE;
+  if (coded && (!k_scale || !v_scale)) return PKV_ERR_ARG;
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(slot_mapping, 8) || !aligned(k_scale, 4) || !aligned(v_scale, 4) ||
       !aligned(err_flag, 4))
@@ -174,7 +175,8 @@ int pkv_decode_num_splits(int num_seqs, int num_kv_heads, int head_dim, int max_
                           pkv_dtype cache_dt) {
   if (num_seqs < 0 || num_kv_heads <= 0 || max_context_len < 0) return PKV_ERR_ARG;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
-  if (cache_dt != PKV_F32 && cache_dt != PKV_BF16 && cache_dt != PKV_I8) return PKV_ERR_DTYPE;
+  if (cache_dt != PKV_F32 && cache_dt != PKV_BF16 && cache_dt != PKV_I8 && cache_dt != PKV_FP8)
+    return PKV_ERR_DTYPE;
   int s, chunk;
   plan(max_context_len, auto_splits(num_seqs, num_kv_heads, head_dim, max_context_len, cache_dt),
        &s, &chunk);
@@ -211,14 +213,14 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
   if (group > 16) return PKV_ERR_SHAPE;
   if (head_dim != 64 && head_dim != 128) return PKV_ERR_SHAPE;
   if (!pow2_in(block_size, 8, 256)) return PKV_ERR_SHAPE;
-  if (cache_dt == PKV_BF16 || cache_dt == PKV_I8) {
+  if (cache_dt == PKV_BF16 || cache_dt == PKV_I8 || cache_dt == PKV_FP8) {
     if (q_dt != PKV_BF16) return PKV_ERR_DTYPE;
   } else if (cache_dt == PKV_F32) {
     if (q_dt != PKV_F32 && q_dt != PKV_BF16) return PKV_ERR_DTYPE;
   } else {
     return PKV_ERR_DTYPE;
   }
-  if (cache_dt == PKV_I8 && (!k_scale || !v_scale)) return PKV_ERR_ARG;
+  if ((cache_dt == PKV_I8 || cache_dt == PKV_FP8) && (!k_scale || !v_scale)) return PKV_ERR_ARG;
   // INT8 scale rows are fetched with bulk copies, which need 16-byte alignment
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(block_tables, 4) ||

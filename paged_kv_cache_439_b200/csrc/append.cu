@@ -12,7 +12,8 @@
 // mlqm.cn page (quantize_tensor): scale = 127 / max|x| over head_dim,
 // code = clamp(rint(x * scale), -128, 127) in fp32 with round-half-to-even;
 // __fdiv_rn / __fmul_rn keep the division and the product correctly rounded
-// and unfused.  An all-zero row stores codes 0 and scale 1.
+// and unfused.  An all-zero row stores codes 0 and scale 1.  The FP8 variant
+// uses scale = 448 / max|x| and E4M3 codes (see append_fp8_kernel).
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -122,6 +123,81 @@ __global__ void __launch_bounds__(kAppendThreads)
   }
 }
 
+// FP8 (E4M3) variant of the same row rule: scale = 448 / max|x|, codes
+// E4M3(x * scale) with round-to-nearest-even and saturation (hardware cvt);
+// an all-zero row stores codes 0 and scale 1.
+template <typename T, int HD>
+__global__ void __launch_bounds__(kAppendThreads)
+    append_fp8_kernel(const T* __restrict__ k, const T* __restrict__ v,
+                      const int64_t* __restrict__ slot_mapping, int num_tokens, int num_kv_heads,
+                      uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
+                      float* __restrict__ k_scale, float* __restrict__ v_scale, int block_size,
+                      long long num_slots, int* err_flag) {
+  constexpr int E = HD / kWarp;  // elements per lane (2 or 4)
+  const int lane = threadIdx.x % kWarp;
+  const long long row = (long long)blockIdx.x * (kAppendThreads / kWarp) + threadIdx.x / kWarp;
+  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
+  if (row >= rows) return;
+  const int t = (int)(row / (2 * num_kv_heads));
+  const int rem = (int)(row % (2 * num_kv_heads));
+  const bool is_v = rem >= num_kv_heads;
+  const int h = is_v ? rem - num_kv_heads : rem;
+  const long long slot = slot_mapping[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (lane == 0 && h == 0 && !is_v) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
+    return;
+  }
+  const T* src = (is_v ? v : k) + ((size_t)t * num_kv_heads + h) * HD + lane * E;
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = to_f32(src[e]);
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float scale = (amax > 0.f) ? __fdiv_rn(448.0f, amax) : 1.0f;
+  uint32_t packed = 0;
+  if (amax > 0.f) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+      packed |= f32x2_to_e4m3x2(__fmul_rn(x[e], scale), __fmul_rn(x[e + 1], scale)) << (8 * e);
+  }
+  const long long blk = slot / block_size;
+  const int off = (int)(slot % block_size);
+  uint8_t* dst = (is_v ? v_cache : k_cache) + ((size_t)slot * num_kv_heads + h) * HD + lane * E;
+  if constexpr (E == 4)
+    *reinterpret_cast<uint32_t*>(dst) = packed;
+  else
+    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+  if (lane == 0) {
+    float* sc = is_v ? v_scale : k_scale;
+    sc[((size_t)blk * num_kv_heads + h) * block_size + off] = scale;
+  }
+}
+
+template <typename T>
+cudaError_t launch_fp8(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
+                       int num_kv_heads, int head_dim, void* k_cache, void* v_cache,
+                       float* k_scale, float* v_scale, int block_size, long long num_slots,
+                       int* err_flag, cudaStream_t st) {
+  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
+  const long long per = kAppendThreads / kWarp;
+  const unsigned grid = (unsigned)((rows + per - 1) / per);
+  if (head_dim == 128)
+    append_fp8_kernel<T, 128><<<grid, kAppendThreads, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
+        num_kv_heads, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale,
+        v_scale, block_size, num_slots, err_flag);
+  else
+    append_fp8_kernel<T, 64><<<grid, kAppendThreads, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
+        num_kv_heads, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale,
+        v_scale, block_size, num_slots, err_flag);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_i8(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
                       int num_kv_heads, int head_dim, void* k_cache, void* v_cache,
@@ -152,6 +228,14 @@ cudaError_t launch_append(const void* k, const void* v, const int64_t* slot_mapp
                           cudaStream_t st) {
   if (num_tokens == 0) return cudaSuccess;
   const long long num_slots = (long long)num_blocks * block_size;
+  if (cache_dt == PKV_FP8) {
+    if (in_dt == PKV_BF16)
+      return launch_fp8<__nv_bfloat16>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                       k_cache, v_cache, k_scale, v_scale, block_size,
+                                       num_slots, err_flag, st);
+    return launch_fp8<float>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim, k_cache,
+                             v_cache, k_scale, v_scale, block_size, num_slots, err_flag, st);
+  }
   if (cache_dt == PKV_I8) {
     if (in_dt == PKV_BF16)
       return launch_i8<__nv_bfloat16>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,

@@ -132,6 +132,27 @@ __device__ __forceinline__ uint32_t i8pair_to_f16x2_biased(uint32_t biased) {
   return prmt(biased, 0x64646464u, SEL);
 }
 
+// Two E4M3 codes -> two exact fp16 values (every E4M3 value is an fp16 value).
+// SEL (prmt selector) puts the first code's byte in bits 0-7 and the second's
+// in bits 8-15; the first lands in the low half of the result.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t e4m3pair_to_f16x2(uint32_t x) {
+  const uint32_t pair = prmt(x, 0u, SEL);
+  uint32_t r;
+  asm("{\n .reg .b16 t;\n cvt.u16.u32 t, %1;\n cvt.rn.f16x2.e4m3x2 %0, t;\n}\n"
+      : "=r"(r)
+      : "r"(pair));
+  return r;
+}
+
+// Two fp32 values -> two E4M3 codes (round to nearest even, saturated to
+// +-448); `lo` lands in bits 0-7.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;\n" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ float fast_rcp(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -220,7 +220,8 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 // mma.sync m16n8k16 with fp32 accumulation (16 tokens x 8 q heads per
 // instruction).  P is split into hi + lo halves so the probabilities keep ~16
 // significant bits.  INT8 codes become exact fp16 values in registers; the
-// per-token scales multiply the fp32 scores (K) and P (V).  The codes reach the
+// per-token scales multiply the fp32 scores (K) and P (V).  FP8 (E4M3) codes
+// convert to exact fp16 with cvt.rn.f16x2.e4m3x2.  INT8 codes reach the
 // tensor core as the exact fp16 values code + 1152 (one byte permute per pair,
 // no subtraction); the constant is removed from the fp32 results: 1152 *
 // sum_d q[h][d] from every score, 1152 * sum_t P[t][h] from the output.
@@ -235,15 +236,20 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 #define PKV_I8_STAGES 3
 #endif
 
-template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
+// Cache formats of the mma engine.
+constexpr int kQuantNone = 0;  // bf16 values
+constexpr int kQuantI8 = 1;    // int8 codes, fp32 scale per token per head
+constexpr int kQuantFp8 = 2;   // E4M3 codes, fp32 scale per token per head
+
+template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
 struct MmaCfg {
-  static constexpr int ELEM = I8 ? 1 : 2;
+  static constexpr int ELEM = QM != kQuantNone ? 1 : 2;
   static constexpr int ROWB = HD * ELEM;        // bytes of one token row of one head
   static constexpr int CH = ROWB / 16;          // 16-byte chunks per row: 4, 8 or 16
   static constexpr int RSTEP = kWarp / CH;      // rows one warp-wide copy covers
   static constexpr int PER_LANE = 16 / RSTEP;   // copies per lane per K (or V) tile
   static constexpr int TILE = 16 * ROWB;
-  static constexpr int STAGE = 2 * TILE + (I8 ? 128 : 0);
+  static constexpr int STAGE = 2 * TILE + (ELEM == 1 ? 128 : 0);
   static constexpr int RING = NWARPS * NSTAGES * STAGE;
   static constexpr int GP = NT * 8;
   static constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
@@ -323,14 +329,17 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
   cp_async_commit();
 }
 
-template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
+template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_mma_kernel(const DecodeParams p) {
-  using Cfg = MmaCfg<HD, I8, NT, NWARPS, NSTAGES>;
+  using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
+  constexpr bool I8 = QM == kQuantI8;
+  constexpr bool F8 = QM == kQuantFp8;
+  constexpr bool Q8 = I8 || F8;         // one-byte codes with per-token scales
   constexpr int KS = HD / 16;           // k-steps of the score mma
   constexpr int MT = HD / 16;           // m-tiles (16 head-dim rows) of the PV mma
-  constexpr int KA = I8 ? KS / 2 : KS;  // ldmatrix.x4 per K tile
-  constexpr int VA = I8 ? MT / 2 : MT;  // ldmatrix.x4 per V tile
+  constexpr int KA = Q8 ? KS / 2 : KS;  // ldmatrix.x4 per K tile
+  constexpr int VA = Q8 ? MT / 2 : MT;  // ldmatrix.x4 per V tile
   constexpr int GP = Cfg::GP;
   constexpr int CH = Cfg::CH;
 
@@ -360,11 +369,11 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         uint32_t b0 = 0, b1 = 0;
         if (h < G) {
           const __nv_bfloat16* qr = qb + (size_t)h * HD;
-          if constexpr (!I8) {
+          if constexpr (!Q8) {
             b0 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4);
             b1 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4 + 8);
           } else {
-            // k-slot order of an int8 chunk: slots 2t,2t+1 <- d 16c+4t+{0,1},
+            // k-slot order of a one-byte-code chunk: slots 2t,2t+1 <- d 16c+4t+{0,1},
             // slots 2t+8,2t+9 <- d 16c+4t+{2,3}
             const uint2 raw = *reinterpret_cast<const uint2*>(qr + 16 * ks + 4 * t4);
             const float2 lo = unpack_bf16(raw.x), hi = unpack_bf16(raw.y);
@@ -434,7 +443,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   for (int i = 0; i < KA; ++i) koff[i] = (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16;
 #pragma unroll
   for (int i = 0; i < VA; ++i)
-    voff[i] = I8 ? (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16
+    voff[i] = Q8 ? (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16
                  : (uint32_t)swz<CH>(lm_row_v, 2 * i + lm_ch_v) * 16;
 
   const uint32_t my_ring = smem_u32(ring) + (uint32_t)(warp * NSTAGES * Cfg::STAGE);
@@ -468,7 +477,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       ldmatrix_x4_trans(vS + voff[a], vf[a][0], vf[a][1], vf[a][2], vf[a][3]);
     float ska = 0.f, skb = 0.f, sva = 0.f, svb = 0.f;
     uint32_t dep = 0;
-    if constexpr (I8) {
+    if constexpr (Q8) {
       float mine;
       asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(mine) : "r"(vS + Cfg::TILE + 4 * lane));
       ska = __shfl_sync(0xffffffffu, mine, g);
@@ -501,7 +510,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[nt][q] = acc2[nt][q] = 0.f;
-    if constexpr (!I8) {
+    if constexpr (!Q8) {
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
@@ -512,6 +521,28 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
           else
             mma_bf16(acc[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
                      qf[ks][nt][1]);
+        }
+      }
+    } else if constexpr (F8) {
+#pragma unroll
+      for (int kp = 0; kp < KS / 2; ++kp) {
+        // kf[kp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1); bytes of a
+        // register are d 4t..4t+3 -> slots (2t, 2t+1) and (2t+8, 2t+9)
+        const uint32_t top[2] = {kf[kp][0], kf[kp][2]};
+        const uint32_t bot[2] = {kf[kp][1], kf[kp][3]};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a0 = e4m3pair_to_f16x2<0x0010>(top[h]);
+          const uint32_t a2 = e4m3pair_to_f16x2<0x0032>(top[h]);
+          const uint32_t a1 = e4m3pair_to_f16x2<0x0010>(bot[h]);
+          const uint32_t a3 = e4m3pair_to_f16x2<0x0032>(bot[h]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            if (h)
+              mma_f16(acc2[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
+            else
+              mma_f16(acc[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
+          }
         }
       }
     } else {
@@ -541,7 +572,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     const bool va = (mask >> g) & 1u, vb = (mask >> (g + 8)) & 1u;
     float fa = p.scale_log2, fb = p.scale_log2;
     float pva = 1.f, pvb = 1.f;
-    if constexpr (I8) {
+    if constexpr (Q8) {
       fa = va ? fa * fast_rcp(ska) : 0.f;
       fb = vb ? fb * fast_rcp(skb) : 0.f;
       pva = va ? fast_rcp(sva) : 0.f;
@@ -580,7 +611,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         p_run[nt][1] = p_run[nt][1] * alpha[nt][1] + (q1 + q3);
       }
       uint32_t h01, h23, l01, l23;
-      if constexpr (!I8) {
+      if constexpr (!Q8) {
         h01 = pack_bf16(q0, q1);
         h23 = pack_bf16(q2, q3);
         const float2 f01 = unpack_bf16(h01), f23 = unpack_bf16(h23);
@@ -611,13 +642,33 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     }
 
     // ---- O^T[d][head] += V^T * P^T
-    if constexpr (!I8) {
+    if constexpr (!Q8) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bh[nt][0], bh[nt][1]);
           mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bl[nt][0], bl[nt][1]);
+        }
+      }
+    } else if constexpr (F8) {
+#pragma unroll
+      for (int mp = 0; mp < MT / 2; ++mp) {
+        // vf[mp] transposed: a register holds bytes (t 2t, d 2g) (2t, 2g+1)
+        // (2t+1, 2g) (2t+1, 2g+1); rows m <-> d as in the INT8 case
+        const uint32_t top[2] = {vf[mp][0], vf[mp][2]};
+        const uint32_t bot[2] = {vf[mp][1], vf[mp][3]};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a0 = e4m3pair_to_f16x2<0x0020>(top[h]);
+          const uint32_t a1 = e4m3pair_to_f16x2<0x0031>(top[h]);
+          const uint32_t a2 = e4m3pair_to_f16x2<0x0020>(bot[h]);
+          const uint32_t a3 = e4m3pair_to_f16x2<0x0031>(bot[h]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          }
         }
       }
     } else {
@@ -696,7 +747,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       for (int j = 0; j < 4; ++j) {
         const int m = g + (j >> 1) * 8;  // fragment row
         const int h = nt * 8 + 2 * t4 + (j & 1);
-        const int d = I8 ? 16 * mt + (m < 8 ? 2 * m : 2 * (m - 8) + 1) : 16 * mt + m;
+        const int d = Q8 ? 16 * mt + (m < 8 ? 2 * m : 2 * (m - 8) + 1) : 16 * mt + m;
         s_o[(warp * GP + h) * HD + d] = o[mt][nt][j];
       }
   combine_and_store<HD, NWARPS, GP>(p, c, s_m, s_l, s_o, s_w, s_L);
@@ -873,34 +924,67 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 // ---------------------------------------------------------------------------
 // Split merge: out = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k} over the partials
 // of one (sequence, q head): the shared-prefix slots [0, ws_base) and the
-// splits that hold tokens.  One CTA per (q head, sequence), one thread per
-// head_dim column.
+// splits that hold tokens.  One warp per (q head, sequence): the lanes first
+// turn the log2-sum-exps into weights (in shared memory), then each lane sums
+// four head_dim columns of the weighted partials with 16-byte loads.
+constexpr int kMergeWarps = 4;
+constexpr int kMergeMaxSlots = 256;  // slots per warp held in shared memory at once
+
 template <int HD>
-__global__ void __launch_bounds__(HD) merge_kernel(const DecodeParams p) {
-  const int qh = blockIdx.x, seq = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeParams p) {
+  __shared__ float s_w[kMergeWarps][kMergeMaxSlots];
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int qh = blockIdx.x * kMergeWarps + warp, seq = blockIdx.y;
+  if (qh >= p.num_q_heads) return;
   const int ctx = effective_ctx(p, seq, false);
   const int rest = ctx > p.t_start ? ctx - p.t_start : 0;
   const int n = p.ws_base + (rest + p.chunk - 1) / p.chunk;
   const size_t r = ((size_t)seq * p.num_q_heads + qh) * p.ws_slots;
-  float M = -CUDART_INF_F;
-  for (int k = 0; k < n; ++k) M = fmaxf(M, p.ws_lse[r + k]);
-  float val = 0.f;
-  if (M != -CUDART_INF_F) {
-    float L = 0.f, O = 0.f;
-    for (int k = 0; k < n; ++k) {
-      const float lse = p.ws_lse[r + k];
-      if (lse == -CUDART_INF_F) continue;
-      const float w = exp2f(lse - M);
-      L += w;
-      O += w * p.ws_o[(r + k) * HD + d];
+  float* w = s_w[warp];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float L = 0.f;
+  // slots in rounds of kMergeMaxSlots (one round unless the plan is huge)
+  for (int base = 0; base < n; base += kMergeMaxSlots) {
+    const int cnt = min(n - base, kMergeMaxSlots);
+    float M = -CUDART_INF_F;
+    for (int k = lane; k < n; k += kWarp) M = fmaxf(M, p.ws_lse[r + k]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (M == -CUDART_INF_F) break;
+    for (int k = lane; k < cnt; k += kWarp) {
+      const float lse = p.ws_lse[r + base + k];
+      w[k] = lse == -CUDART_INF_F ? 0.f : exp2f(lse - M);
     }
-    val = O / L;
+    __syncwarp();
+    if (base == 0) L = 0.f;
+    // weights relative to the max over all slots, so rounds add up directly
+    for (int k = 0; k < cnt; ++k) L += w[k];
+    if (lane * 4 < HD) {
+#pragma unroll 4
+      for (int k = 0; k < cnt; ++k) {
+        const float wk = w[k];
+        if (wk == 0.f) continue;
+        const float4 v =
+            *reinterpret_cast<const float4*>(p.ws_o + (r + base + k) * HD + lane * 4);
+        acc[0] += wk * v.x;
+        acc[1] += wk * v.y;
+        acc[2] += wk * v.z;
+        acc[3] += wk * v.w;
+      }
+    }
+    __syncwarp();
   }
-  const size_t o = ((size_t)seq * p.num_q_heads + qh) * HD + d;
-  if (p.out_f32)
-    static_cast<float*>(p.out)[o] = val;
-  else
-    static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(val);
+  if (lane * 4 >= HD) return;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const size_t o = ((size_t)seq * p.num_q_heads + qh) * HD + lane * 4;
+  if (p.out_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  } else {
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(p.out) + o;
+    *reinterpret_cast<uint2*>(ob) =
+        make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -935,11 +1019,11 @@ cudaError_t prepare(int smem) {
   return e;
 }
 
-template <int HD, bool I8, int NT, int NWARPS, int NSTAGES>
+template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = MmaCfg<HD, I8, NT, NWARPS, NSTAGES>;
+  using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
   const int smem = p.phys_bytes + Cfg::BODY;
-  constexpr auto k = decode_mma_kernel<HD, I8, NT, NWARPS, NSTAGES>;
+  constexpr auto k = decode_mma_kernel<HD, QM, NT, NWARPS, NSTAGES>;
   cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
@@ -984,20 +1068,23 @@ int occupancy(int threads, int smem) {
 
 constexpr int kTypicalPhysBytes = 1024;  // block-table slice of a typical split
 
-template <int HD, bool I8>
+template <int HD, int QM>
 int mma_occupancy() {
-  using Cfg = MmaCfg<HD, I8, 1, kMW, I8 ? PKV_I8_STAGES : PKV_BF16_STAGES>;
-  return occupancy<decode_mma_kernel<HD, I8, 1, kMW, I8 ? PKV_I8_STAGES : PKV_BF16_STAGES>>(
-      kMW * kWarp, kTypicalPhysBytes + Cfg::BODY);
+  constexpr int NS = QM != kQuantNone ? PKV_I8_STAGES : PKV_BF16_STAGES;
+  using Cfg = MmaCfg<HD, QM, 1, kMW, NS>;
+  return occupancy<decode_mma_kernel<HD, QM, 1, kMW, NS>>(kMW * kWarp,
+                                                          kTypicalPhysBytes + Cfg::BODY);
 }
 
 }  // namespace
 
 int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim) {
-  if (cache_dt == PKV_BF16) return head_dim == 128 ? mma_occupancy<128, false>()
-                                                   : mma_occupancy<64, false>();
-  if (cache_dt == PKV_I8) return head_dim == 128 ? mma_occupancy<128, true>()
-                                                 : mma_occupancy<64, true>();
+  if (cache_dt == PKV_BF16) return head_dim == 128 ? mma_occupancy<128, kQuantNone>()
+                                                   : mma_occupancy<64, kQuantNone>();
+  if (cache_dt == PKV_I8) return head_dim == 128 ? mma_occupancy<128, kQuantI8>()
+                                                 : mma_occupancy<64, kQuantI8>();
+  if (cache_dt == PKV_FP8) return head_dim == 128 ? mma_occupancy<128, kQuantFp8>()
+                                                  : mma_occupancy<64, kQuantFp8>();
   const int smem = kF32Warps * kF32Stages * 2 * 16 * head_dim * 4 + 16 * head_dim * 4 + 1024;
   const int n = (228 * 1024) / (smem + 1024);
   return n < 1 ? 1 : n;
@@ -1009,28 +1096,35 @@ cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_di
   const bool two = p.group > 8;
   if (cache_dt == PKV_BF16) {
     if (head_dim == 128)
-      return two ? launch_mma<128, false, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
-                 : launch_mma<128, false, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
-    return two ? launch_mma<64, false, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
-               : launch_mma<64, false, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
+      return two ? launch_mma<128, kQuantNone, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
+                 : launch_mma<128, kQuantNone, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
+    return two ? launch_mma<64, kQuantNone, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
+               : launch_mma<64, kQuantNone, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
   }
   if (cache_dt == PKV_I8) {
     if (head_dim == 128)
-      return two ? launch_mma<128, true, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-                 : launch_mma<128, true, 1, kMW, PKV_I8_STAGES>(p, grid, st);
-    return two ? launch_mma<64, true, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-               : launch_mma<64, true, 1, kMW, PKV_I8_STAGES>(p, grid, st);
+      return two ? launch_mma<128, kQuantI8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+                 : launch_mma<128, kQuantI8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
+    return two ? launch_mma<64, kQuantI8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+               : launch_mma<64, kQuantI8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
+  }
+  if (cache_dt == PKV_FP8) {
+    if (head_dim == 128)
+      return two ? launch_mma<128, kQuantFp8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+                 : launch_mma<128, kQuantFp8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
+    return two ? launch_mma<64, kQuantFp8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
+               : launch_mma<64, kQuantFp8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
   }
   if (head_dim == 128) return launch_simt<128, kF32Warps, kF32Stages>(p, grid, st);
   return launch_simt<64, kF32Warps, kF32Stages>(p, grid, st);
 }
 
 cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st) {
-  dim3 grid(p.num_q_heads, p.num_seqs);
+  dim3 grid((p.num_q_heads + kMergeWarps - 1) / kMergeWarps, p.num_seqs);
   if (head_dim == 128)
-    merge_kernel<128><<<grid, 128, 0, st>>>(p);
+    merge_kernel<128><<<grid, kMergeWarps * kWarp, 0, st>>>(p);
   else
-    merge_kernel<64><<<grid, 64, 0, st>>>(p);
+    merge_kernel<64><<<grid, kMergeWarps * kWarp, 0, st>>>(p);
   return cudaGetLastError();
 }
 

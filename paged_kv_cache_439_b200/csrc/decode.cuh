@@ -44,7 +44,7 @@ struct PrefixParams {
   int rows;           // q rows per KV head: num_seqs * group
   int phys_bytes;     // shared-memory bytes for one slice's block-table entries
 };
-constexpr int kPrefixWarps = 8;    // 16 q rows per warp
+constexpr int kPrefixWarps = 4;    // 16 q rows per warp
 constexpr int kPrefixTokens = 64;  // tokens per shared-memory stage
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,

@@ -151,9 +151,17 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       cp_async_commit();
   }
 
-  // ldmatrix lane addressing (matrix j = lane / 8 supplies its row lane % 8)
+  // ldmatrix lane addressing (matrix j = lane / 8 supplies its row lane % 8).
+  // A row 16 * j + r of a stage has the swizzle of row r (16 * j keeps r & 7),
+  // so the per-lane offsets inside a 16-token tile are fixed.
   const int kr = (lane & 7) + ((lane >> 4) & 1) * 8, kc = (lane >> 3) & 1;  // K: b0,b1 of 2 n-tiles
   const int vr = (lane & 7) + ((lane >> 3) & 1) * 8, vc = lane >> 4;        // V^T: 2 n-tiles
+  uint32_t koff[KS], voff[NTD / 2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) koff[ks] = (uint32_t)swz<CH>(kr, 2 * ks + kc) * 16;
+#pragma unroll
+  for (int dp = 0; dp < NTD / 2; ++dp) voff[dp] = (uint32_t)swz<CH>(vr, 2 * dp + vc) * 16;
+  constexpr uint32_t kTileBytes = 16 * Cfg::ROWB;  // one 16-token tile of K (or V)
 
   for (int s = 0; s < nst; ++s) {
     {
@@ -176,24 +184,33 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       const bool tv = tl < t1 && s_phys[(tl >> p.log2_bs) - blk0] >= 0;
       const uint32_t tmask = __ballot_sync(0xffffffffu, tv) & 0xFFFFu;
 
-      // ---- S[row][token] = Q K^T, two 8-token n-tiles
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // ---- S[row][token] = Q K^T, two 8-token n-tiles (even and odd k-steps in
+      // separate accumulators to halve the dependent mma chains)
+      float acc[2][2][4] = {};
+      const uint32_t kT = kS + (uint32_t)j * kTileBytes;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t b0, b1, b2, b3;  // (tok 0-7, c) (tok 0-7, c+1) (tok 8-15, c) (tok 8-15, c+1)
-        ldmatrix_x4(kS + (uint32_t)swz<CH>(16 * j + kr, 2 * ks + kc) * 16, b0, b1, b2, b3);
-        mma_bf16(acc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-        mma_bf16(acc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+        ldmatrix_x4(kT + koff[ks], b0, b1, b2, b3);
+        mma_bf16(acc[ks & 1][0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+        mma_bf16(acc[ks & 1][1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
       }
       // ---- mask, online softmax per row (rows g, g + 8; tokens 8nt + 2t4 + e)
+      const bool full = __all_sync(0xffffffffu, tmask == 0xFFFFu && tj + 16 <= lim[0] &&
+                                                    tj + 16 <= lim[1]);
       float sv[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int col = 8 * nt + 2 * t4 + (e & 1);
-          const bool ok = ((tmask >> col) & 1u) && (tj + col < lim[e >> 1]);
-          sv[nt][e] = ok ? acc[nt][e] * p.scale_log2 : -CUDART_INF_F;
+          const float x = (acc[0][nt][e] + acc[1][nt][e]) * p.scale_log2;
+          if (full) {
+            sv[nt][e] = x;
+          } else {
+            const int col = 8 * nt + 2 * t4 + (e & 1);
+            const bool ok = ((tmask >> col) & 1u) && (tj + col < lim[e >> 1]);
+            sv[nt][e] = ok ? x : -CUDART_INF_F;
+          }
         }
       float alpha[2];
       bool rescale = false;
@@ -243,7 +260,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
       for (int dp = 0; dp < NTD / 2; ++dp) {
         uint32_t b0, b1, b2, b3;  // (tok 0-7, c) (tok 8-15, c) (tok 0-7, c+1) (tok 8-15, c+1)
-        ldmatrix_x4_trans(vS + (uint32_t)swz<CH>(16 * j + vr, 2 * dp + vc) * 16, b0, b1, b2, b3);
+        ldmatrix_x4_trans(vS + (uint32_t)j * kTileBytes + voff[dp], b0, b1, b2, b3);
         mma_bf16(o[2 * dp], ph[0], ph[1], ph[2], ph[3], b0, b1);
         mma_bf16(o[2 * dp], pl[0], pl[1], pl[2], pl[3], b0, b1);
         mma_bf16(o[2 * dp + 1], ph[0], ph[1], ph[2], ph[3], b2, b3);

@@ -89,7 +89,7 @@ class Workload:
     head_dim: int
     block_size: int
     num_blocks: int
-    cache_dtype: str            # "f32" | "bf16" | "i8"
+    cache_dtype: str            # "f32" | "bf16" | "i8" | "fp8"
     input_dtype: torch.dtype    # dtype of q and of the K/V rows to append
     softmax_scale: float
     context_lens: torch.Tensor  # int32 [B]
@@ -117,13 +117,13 @@ class Workload:
         return self.num_q_heads // self.num_kv_heads
 
     def cache_elem_bytes(self) -> int:
-        return {"f32": 4, "bf16": 2, "i8": 1}[self.cache_dtype]
+        return {"f32": 4, "bf16": 2, "i8": 1, "fp8": 1}[self.cache_dtype]
 
     def kv_bytes(self) -> int:
         """Algorithmic KV bytes one decode call reads (K and V, plus INT8 scales)."""
         toks = int(self.context_lens.to(torch.int64).sum().item())
         per_tok_head = 2 * self.head_dim * self.cache_elem_bytes()
-        if self.cache_dtype == "i8":
+        if self.cache_dtype in ("i8", "fp8"):
             per_tok_head += 2 * 4
         return toks * self.num_kv_heads * per_tok_head
 
@@ -149,7 +149,7 @@ def make_custom(name: str, context_lens: List[int], num_q_heads: int, num_kv_hea
     prefix tokens are pre-filled once.  ``context_lens`` then counts prefix
     plus suffix.
     """
-    if cache_dtype not in ("f32", "bf16", "i8"):
+    if cache_dtype not in ("f32", "bf16", "i8", "fp8"):
         raise ValueError(cache_dtype)
     if num_q_heads % num_kv_heads:
         raise ValueError("num_q_heads must be a multiple of num_kv_heads")

@@ -45,9 +45,10 @@ class OracleCache:
     def __init__(self, wl: Workload):
         self.wl = wl
         shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
-        if wl.cache_dtype == "i8":
-            self.k = np.full(shape, 127, np.int8)
-            self.v = np.full(shape, 127, np.int8)
+        if wl.cache_dtype in ("i8", "fp8"):
+            dt = np.int8 if wl.cache_dtype == "i8" else np.uint8
+            self.k = np.full(shape, 127, dt)
+            self.v = np.full(shape, 127, dt)
             sshape = (wl.num_blocks, wl.num_kv_heads, wl.block_size)
             self.ks = np.full(sshape, np.nan, np.float32)
             self.vs = np.full(sshape, np.nan, np.float32)
@@ -65,6 +66,9 @@ class OracleCache:
             vf = v.float().numpy()
             oracle.append_int8(kf, sl, self.k, self.ks)
             oracle.append_int8(vf, sl, self.v, self.vs)
+        elif self.wl.cache_dtype == "fp8":
+            oracle.append_fp8(k.float().numpy(), sl, self.k, self.ks)
+            oracle.append_fp8(v.float().numpy(), sl, self.v, self.vs)
         else:
             oracle.append_rows(host_rows(k), sl, self.k)
             oracle.append_rows(host_rows(v), sl, self.v)
@@ -82,6 +86,9 @@ class OracleCache:
         if wl.cache_dtype == "i8":
             return oracle.paged_decode_i8(q, self.k, self.v, self.ks, self.vs, bt, cl,
                                           wl.softmax_scale, threads)
+        if wl.cache_dtype == "fp8":
+            return oracle.paged_decode_fp8(q, self.k, self.v, self.ks, self.vs, bt, cl,
+                                           wl.softmax_scale, threads)
         if wl.cache_dtype == "bf16":
             return oracle.paged_decode(q, widen_bf16(self.k), widen_bf16(self.v), bt, cl,
                                        wl.softmax_scale, threads)
@@ -90,7 +97,8 @@ class OracleCache:
 
 # ---------------------------------------------------------------- CUDA side
 
-_TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8}
+_TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8,
+             "fp8": torch.float8_e4m3fn}
 
 
 class GpuCache:
@@ -103,9 +111,9 @@ class GpuCache:
         self.device = device
         shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
         dt = _TORCH_DT[wl.cache_dtype]
-        if wl.cache_dtype == "i8":
-            self.k = torch.full(shape, 127, dtype=dt, device=device)
-            self.v = torch.full(shape, 127, dtype=dt, device=device)
+        if wl.cache_dtype in ("i8", "fp8"):
+            self.k = torch.full(shape, 127, dtype=torch.int8, device=device).view(dt)
+            self.v = torch.full(shape, 127, dtype=torch.int8, device=device).view(dt)
             sshape = (wl.num_blocks, wl.num_kv_heads, wl.block_size)
             self.ks = torch.full(sshape, float("nan"), dtype=torch.float32, device=device)
             self.vs = torch.full(sshape, float("nan"), dtype=torch.float32, device=device)
@@ -172,6 +180,8 @@ def bits(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).numpy()
     if t.dtype == torch.float32:
         return t.view(torch.int32).numpy()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
     return t.numpy()
 
 

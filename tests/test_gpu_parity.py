@@ -31,7 +31,8 @@ def _wl(cache_dtype, nq, nkv, d, bs, lens=RAGGED, seed=11, **kw):
 # ---------------------------------------------------------------- append
 
 @pytest.mark.parametrize("cache_dtype,d,bs", [("f32", 64, 16), ("bf16", 128, 16),
-                                              ("bf16", 64, 8), ("i8", 128, 16), ("i8", 64, 256)])
+                                              ("bf16", 64, 8), ("i8", 128, 16), ("i8", 64, 256),
+                                              ("fp8", 128, 16), ("fp8", 64, 8)])
 def test_append_bit_exact(cache_dtype, d, bs):
     wl = _wl(cache_dtype, 8, 4, d, bs, lens=[1, 40, 300], outlier_prob=0.01)
     g = GpuCache(wl).fill()
@@ -39,7 +40,7 @@ def test_append_bit_exact(cache_dtype, d, bs):
     torch.cuda.synchronize()
     assert np.array_equal(bits(g.k), oracle_bits(wl, o.k))
     assert np.array_equal(bits(g.v), oracle_bits(wl, o.v))
-    if cache_dtype == "i8":
+    if cache_dtype in ("i8", "fp8"):
         assert np.array_equal(bits(g.ks), o.ks.view(np.int32))
         assert np.array_equal(bits(g.vs), o.vs.view(np.int32))
     assert g.flags() == 0
@@ -83,13 +84,15 @@ def test_tiny_workload(splits):
     assert g.flags() == 0
 
 
-GRID = [(dt, g, d) for dt in ("bf16", "i8", "f32") for g in (1, 4, 8, 16) for d in (64, 128)]
+GRID = [(dt, g, d) for dt in ("bf16", "i8", "fp8", "f32") for g in (1, 4, 8, 16)
+        for d in (64, 128)]
 
 
 @pytest.mark.parametrize("cache_dtype,group,d", GRID)
 def test_decode_dtype_group_headdim(cache_dtype, group, d):
     nkv = 2
-    wl = _wl(cache_dtype, nkv * group, nkv, d, 16, outlier_prob=0.01 if cache_dtype == "i8" else 0)
+    wl = _wl(cache_dtype, nkv * group, nkv, d, 16,
+             outlier_prob=0.01 if cache_dtype in ("i8", "fp8") else 0)
     g = GpuCache(wl).fill()
     ref = OracleCache(wl).fill().decode()
     for splits in (0, 1, 5):
@@ -99,7 +102,8 @@ def test_decode_dtype_group_headdim(cache_dtype, group, d):
 
 
 @pytest.mark.parametrize("cache_dtype,bs", [("bf16", 8), ("bf16", 32), ("bf16", 256),
-                                            ("i8", 8), ("i8", 256), ("f32", 128)])
+                                            ("i8", 8), ("i8", 256), ("fp8", 8), ("fp8", 256),
+                                            ("f32", 128)])
 def test_decode_block_sizes(cache_dtype, bs):
     wl = _wl(cache_dtype, 16, 2, 128, bs)
     g = GpuCache(wl).fill()
@@ -128,7 +132,7 @@ def test_mqa_single_kv_head():
 
 # ---------------------------------------------------------------- invariants
 
-@pytest.mark.parametrize("cache_dtype", ["bf16", "i8"])
+@pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8"])
 def test_block_permutation_gives_bit_identical_output(cache_dtype):
     a = _wl(cache_dtype, 32, 4, 128, 16, placement_seed=1)
     b = _wl(cache_dtype, 32, 4, 128, 16, placement_seed=2)
@@ -220,14 +224,15 @@ def test_error_status_from_binding():
 
 # ---------------------------------------------------------------- full-size workloads
 
-FULL = [("llama2-7b-mha", None), ("llama2-70b-gqa", None), ("llama2-13b-int8", None),
-        ("shared-prefix", 16), ("shared-prefix", 256)]
+FULL = [("llama2-7b-mha", None, None), ("llama2-70b-gqa", None, None),
+        ("llama2-13b-int8", None, None), ("llama2-13b-int8", None, "fp8"),
+        ("shared-prefix", 16, None), ("shared-prefix", 256, None)]
 
 
-@pytest.mark.parametrize("name,bs", FULL)
-def test_full_workload_parity(name, bs):
+@pytest.mark.parametrize("name,bs,kv", FULL)
+def test_full_workload_parity(name, bs, kv):
     """The workloads at full size, in the launch configuration the benchmark times."""
-    wl = make_workload(name, block_size=bs)
+    wl = make_workload(name, block_size=bs, **({"cache_dtype": kv} if kv else {}))
     g = GpuCache(wl).fill()
     out = g.decode(num_splits=0)
     torch.cuda.synchronize()

@@ -381,3 +381,78 @@ def test_workload_tiny_through_oracle_matches_sdpa():
     ref = _sdpa_reference(wl.q.numpy(), kc, vc, tables, cl, wl.softmax_scale, bs)
     assert np.isfinite(got).all()           # NaN-poisoned slots were never read
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3)
+
+def _torch_e4m3_value(code):
+    return float(torch.tensor([code], dtype=torch.uint8).view(torch.float8_e4m3fn).float()[0])
+
+
+def test_e4m3_decode_matches_library_for_all_codes():
+    for code in range(256):
+        ours = oracle.e4m3_decode(code)
+        ref = _torch_e4m3_value(code)
+        if math.isnan(ref):
+            assert math.isnan(ours) and (code & 0x7F) == 0x7F
+        else:
+            assert ours == ref, (code, ours, ref)
+    assert oracle.e4m3_decode(0x7E) == 448.0 and oracle.e4m3_decode(0x01) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_library_rounding():
+    rng = np.random.default_rng(12)
+    xs = np.concatenate([rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 0.01,
+                         rng.standard_normal(2000) * 30]).astype(np.float32)
+    # exact midpoints between neighbouring finite values (ties -> even mantissa)
+    vals = sorted({oracle.e4m3_decode(c) for c in range(0x7F) if not math.isnan(oracle.e4m3_decode(c))})
+    mids = np.array([(a + b) / 2 for a, b in zip(vals, vals[1:])], dtype=np.float32)
+    xs = np.concatenate([xs, mids, -mids])
+    xs = xs[np.abs(xs) <= 448]
+    ref = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = np.array([oracle.e4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    # +-0 encode as the same magnitude
+    assert np.array_equal(ours & 0x7F, ref & 0x7F)
+    nz = (ref & 0x7F) != 0
+    assert np.array_equal(ours[nz], ref[nz])
+
+
+def test_e4m3_saturates_and_quantize_fp8_rules():
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_encode(-500.0) == 0xFE
+    assert oracle.e4m3_encode(448.0001) == 0x7E
+    rng = np.random.default_rng(13)
+    for _ in range(100):
+        x = rng.standard_normal(128).astype(np.float32)
+        x[rng.random(128) < 0.02] *= 8
+        codes, s = oracle.quantize_row_fp8(x)
+        assert s == np.float32(np.float32(448.0) / np.float32(np.abs(x).max()))
+        i = int(np.argmax(np.abs(x)))
+        assert codes[i] == (0x7E if x[i] > 0 else 0xFE)          # absmax -> +-448
+        dq = np.array([oracle.e4m3_decode(c) for c in codes]) / float(s)
+        # half a quantum: 2^-4 relative for normals, 2^-10 absolute (scaled) below
+        bound = np.maximum(np.abs(x.astype(np.float64)) * 2.0 ** -4, 2.0 ** -10 / float(s))
+        assert (np.abs(dq - x) <= bound * (1 + 1e-6)).all()
+    codes, s = oracle.quantize_row_fp8(np.zeros(8, np.float32))
+    assert s == np.float32(1.0) and (codes == 0).all()
+
+
+def test_fp8_decode_equals_attention_on_dequantised_values():
+    rng = np.random.default_rng(14)
+    bs, nkv, d = 16, 2, 32
+    q, kf, vf, tables, cl = _random_paged(rng, [5, 17, 40], 4, nkv, d, bs)
+    nb = kf.shape[0]
+    kc = np.zeros((nb, bs, nkv, d), np.uint8)
+    vc = np.zeros_like(kc)
+    ks = np.ones((nb, nkv, bs), np.float32)
+    vs = np.ones_like(ks)
+    slots = np.arange(nb * bs, dtype=np.int64)
+    oracle.append_fp8(kf.reshape(-1, nkv, d), slots, kc, ks)
+    oracle.append_fp8(vf.reshape(-1, nkv, d), slots, vc, vs)
+    got = oracle.paged_decode_fp8(q, kc, vc, ks, vs, tables, cl, 0.25)
+    table = np.array([oracle.e4m3_decode(c) for c in range(256)])
+    kd = table[kc] / ks.transpose(0, 2, 1)[..., None].astype(np.float64)
+    vd = table[vc] / vs.transpose(0, 2, 1)[..., None].astype(np.float64)
+    ref = _sdpa_reference(q, kd, vd, tables, cl, 0.25, bs)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    plain = oracle.paged_decode(q, kf, vf, tables, cl, 0.25)
+    assert np.abs(got - plain).max() < 0.2
