@@ -10,6 +10,7 @@ the timed region.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python -m torch.distributed.run --nproc-per-node N ... bench.py --gpus N
     python bench.py --impl reference      # the CPU oracle, same metric and config
+    python bench.py --swap                # block swap out/in through pinned host memory
 
 Prints one JSON line (rank 0).  ``value`` is KV bytes read by the decode
 calls of all ranks divided by the max-over-ranks device time of the K timed
@@ -56,6 +57,9 @@ def parse():
                     help="override the workload's KV-cache format")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix workload: read the shared blocks once per KV head")
+    ap.add_argument("--swap", action="store_true",
+                    help="time swapping every sequence's blocks out to pinned host memory and "
+                         "back (pkv_copy_blocks) against a plain pinned memcpy of the same bytes")
     return ap.parse_args()
 
 
@@ -270,10 +274,102 @@ def config_dict(wl, args, splits):
 
 # ---------------------------------------------------------------- GPU arm
 
+def device_cache(wl, dev):
+    """The workload's paged cache on the device, pre-filled through the C ABI."""
+    import torch
+    import paged_kv_cache_439_b200 as pkv
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8,
+           "fp8": torch.float8_e4m3fn}[wl.cache_dtype]
+    shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
+    k_cache = torch.zeros(shape, dtype=torch.uint8 if tdt == torch.float8_e4m3fn else tdt,
+                          device=dev).view(tdt)
+    v_cache = torch.zeros_like(k_cache)
+    k_scale = v_scale = None
+    if wl.cache_dtype in ("i8", "fp8"):
+        sshape = (wl.num_blocks, wl.num_kv_heads, wl.block_size)
+        k_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
+        v_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    pk, pv, ps = (wl.prefill_k.to(dev), wl.prefill_v.to(dev), wl.prefill_slots.to(dev))
+    CH = 1 << 16
+    for i in range(0, pk.shape[0], CH):
+        pkv.kv_cache_append(pk[i:i + CH], pv[i:i + CH], ps[i:i + CH], k_cache, v_cache, k_scale,
+                            v_scale, err_flag=err)
+    return tdt, k_cache, v_cache, k_scale, v_scale, err
+
+
+def run_swap(args):
+    """Swap bandwidth: every block of every sequence out to a pinned host pool
+    in one pkv_copy_blocks launch, then back in, each timed with CUDA events;
+    the plain pinned cudaMemcpyAsync of the same byte count in each direction
+    is the link's measured peak."""
+    import torch
+    import paged_kv_cache_439_b200 as pkv
+    from paged_kv_cache_439_b200.workloads import make_workload, workload_seed
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    extra = {"cache_dtype": args.kv_dtype} if args.kv_dtype else {}
+    wl = make_workload(args.workload, block_size=args.block_size,
+                       data_seed=workload_seed(args.workload), **extra)
+    _, k, v, ks, vs, err = device_cache(wl, dev)
+    used = list(dict.fromkeys(wl.block_tables[wl.block_tables >= 0].tolist()))
+    n = len(used)
+    hk = torch.empty((n,) + tuple(k.shape[1:]), dtype=k.dtype).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    hks = hvs = None
+    if ks is not None:
+        hks = torch.empty((n,) + tuple(ks.shape[1:]), dtype=ks.dtype).pin_memory()
+        hvs = torch.empty_like(hks).pin_memory()
+    out_pairs = torch.tensor([[b, i] for i, b in enumerate(used)], dtype=torch.int32, device=dev)
+    in_pairs = out_pairs.flip(1).contiguous()
+    nbytes = 2 * (hk.numel() * hk.element_size() + (hks.numel() * 4 if hks is not None else 0))
+    flat_dev = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    flat_host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    reps = max(1, min(args.steps, 20))
+    t_out = timed(lambda: pkv.copy_blocks(hk, hv, k, v, out_pairs, hks, hvs, ks, vs,
+                                          err_flag=err), reps)
+    t_in = timed(lambda: pkv.copy_blocks(k, v, hk, hv, in_pairs, ks, vs, hks, hvs,
+                                         err_flag=err), reps)
+    t_d2h = timed(lambda: flat_host.copy_(flat_dev, non_blocking=True), reps)
+    t_h2d = timed(lambda: flat_dev.copy_(flat_host, non_blocking=True), reps)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"copy kernel flagged {int(err.item())}")
+    gbs = lambda ms: nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": "KV block swap GB/s (device<->pinned host, one launch per direction)",
+            "value": round(min(gbs(t_out), gbs(t_in)), 2), "unit": "GB/s", "n_gpus": 1,
+            "steps": reps, "warmup": 3, "higher_is_better": True,
+            "config": {"workload": wl.name, "cache_dtype": wl.cache_dtype, "blocks": n,
+                       "bytes_per_direction": nbytes},
+            "swap_out_gbs": round(gbs(t_out), 2), "swap_in_gbs": round(gbs(t_in), 2),
+            "memcpy_d2h_gbs": round(gbs(t_d2h), 2), "memcpy_h2d_gbs": round(gbs(t_h2d), 2),
+            "frac_out": round(t_d2h / t_out, 3), "frac_in": round(t_h2d / t_in, 3)}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.swap:
+        run_swap(args)
         return
     import torch
     import torch.distributed as dist
@@ -296,26 +392,7 @@ def main():
     extra = {"cache_dtype": args.kv_dtype} if args.kv_dtype else {}
     wl = make_workload(args.workload, block_size=args.block_size,
                        data_seed=pdist.replica_seed(workload_seed(args.workload), rank), **extra)
-    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "i8": torch.int8,
-           "fp8": torch.float8_e4m3fn}[wl.cache_dtype]
-    shape = (wl.num_blocks, wl.block_size, wl.num_kv_heads, wl.head_dim)
-    k_cache = torch.zeros(shape, dtype=torch.uint8 if tdt == torch.float8_e4m3fn else tdt,
-                          device=dev).view(tdt)
-    v_cache = torch.zeros_like(k_cache)
-    k_scale = v_scale = None
-    if wl.cache_dtype in ("i8", "fp8"):
-        sshape = (wl.num_blocks, wl.num_kv_heads, wl.block_size)
-        k_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
-        v_scale = torch.ones(sshape, dtype=torch.float32, device=dev)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-
-    # pre-fill (not timed)
-    pk, pv, ps = (wl.prefill_k.to(dev), wl.prefill_v.to(dev), wl.prefill_slots.to(dev))
-    CH = 1 << 16
-    for i in range(0, pk.shape[0], CH):
-        pkv.kv_cache_append(pk[i:i + CH], pv[i:i + CH], ps[i:i + CH], k_cache, v_cache, k_scale,
-                            v_scale, err_flag=err)
-    del pk, pv, ps
+    tdt, k_cache, v_cache, k_scale, v_scale, err = device_cache(wl, dev)
 
     q = wl.q.to(dev)
     nk, nv, ns = wl.new_k.to(dev), wl.new_v.to(dev), wl.new_slots.to(dev)

@@ -54,7 +54,8 @@ typedef enum {
   PKV_ERR_WORKSPACE = -5,   /* split-K needs a workspace of pkv_workspace_size() bytes */
   PKV_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
   PKV_ERR_ALIGN = -7,       /* a device pointer is not 16-byte aligned */
-  PKV_ERR_SCRATCH_LIMIT = -8 /* split-K scratch would exceed PKV_NOALLOC_SCRATCH_BYTES */
+  PKV_ERR_SCRATCH_LIMIT = -8, /* split-K scratch would exceed PKV_NOALLOC_SCRATCH_BYTES */
+  PKV_ERR_NO_BLOCKS = -9      /* the block pool cannot supply the blocks an operation needs */
 } pkv_status;
 
 /* Bits written into *err_flag by the kernels. */
@@ -224,6 +225,75 @@ int pkv_paged_attention_decode_noalloc(void* out, const void* q, pkv_dtype q_dt,
                                        int num_kv_heads, int head_dim, int block_size,
                                        int num_blocks, float softmax_scale, int num_splits,
                                        int* err_flag, pkv_stream_t stream);
+
+/*
+ * Block manager (host) - the pages' block bookkeeping ([mlqm] §2: fixed-size
+ * blocks, a block table from logical to physical blocks, Block.ref_count;
+ * [yunthe], PagedAttention section: blocks allocated on demand, reclaimed when
+ * a sequence ends; its deployment parameters: swap_space moves inactive KV to
+ * CPU memory).  A manager owns the ids of one pool of num_blocks blocks
+ * (device or host); the caller owns the memory and moves data with
+ * pkv_copy_blocks.  Blocks come off a free list (block 0 first, freed blocks
+ * reused last-in first-out).  Every call is atomic (PKV_ERR_NO_BLOCKS leaves
+ * the manager unchanged) and calls on one manager are serialised by a mutex.
+ * Sequence ids are caller-chosen 64-bit keys.
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+int pkv_bm_create(int num_blocks, int block_size, pkv_block_manager** out);
+void pkv_bm_destroy(pkv_block_manager* m);
+/* free blocks; references of a block (0 = free) */
+int pkv_bm_num_free(pkv_block_manager* m);
+int pkv_bm_ref_count(pkv_block_manager* m, int32_t block);
+/* a new empty sequence */
+int pkv_bm_add_sequence(pkv_block_manager* m, int64_t seq_id);
+/* child shares every block of parent (references + 1) and its length */
+int pkv_bm_fork(pkv_block_manager* m, int64_t parent, int64_t child);
+/* blocks pkv_bm_reserve would take for num_tokens more tokens (>= 0) */
+int pkv_bm_blocks_needed(pkv_block_manager* m, int64_t seq_id, int num_tokens);
+/*
+ * Reserves the slots of the sequence's next num_tokens tokens (slots_out[i] =
+ * block * block_size + offset, ready for pkv_kv_cache_append), allocating a
+ * block at each block boundary.  If the sequence's last block is shared and
+ * partially filled it is first replaced by a private block (copy-on-write):
+ * *num_cow = 1 and cow_pair_out[0..1] = (shared block, new block) - copy it
+ * with pkv_copy_blocks before appending.  Otherwise *num_cow = 0.
+ */
+int pkv_bm_reserve(pkv_block_manager* m, int64_t seq_id, int num_tokens, int64_t* slots_out,
+                   int32_t* cow_pair_out, int* num_cow);
+/* drops the sequence; blocks whose references reach 0 return to the free list */
+int pkv_bm_free(pkv_block_manager* m, int64_t seq_id);
+int pkv_bm_seq_len(pkv_block_manager* m, int64_t seq_id, int64_t* len_out, int* num_blocks_out);
+/* dense block tables [num_seqs][max_blocks_per_seq] (padding -1) and lengths */
+int pkv_bm_block_tables(pkv_block_manager* m, const int64_t* seq_ids, int num_seqs,
+                        int max_blocks_per_seq, int32_t* tables_out, int32_t* lens_out);
+/*
+ * Moves a sequence between a device-pool manager and a host-pool manager (same
+ * block_size): fresh blocks are taken in the destination, the source blocks
+ * are released, and pairs_out[2i], pairs_out[2i+1] = (source block, destination
+ * block) for each of its *num_pairs blocks, in table order - pass them to
+ * pkv_copy_blocks.  A block the sequence shared with others stays with them.
+ */
+int pkv_bm_swap_out(pkv_block_manager* device, pkv_block_manager* host, int64_t seq_id,
+                    int32_t* pairs_out, int capacity, int* num_pairs);
+int pkv_bm_swap_in(pkv_block_manager* host, pkv_block_manager* device, int64_t seq_id,
+                   int32_t* pairs_out, int capacity, int* num_pairs);
+
+/*
+ * pkv_copy_blocks - copies whole blocks: for each pair i, block pairs[2i] of the
+ * source pool goes to block pairs[2i+1] of the destination pool, K and V (and
+ * the per-token scales when scale_bytes_per_block > 0).  Pools are laid out as
+ * the cache ([num_blocks][block_bytes]) and may be device memory or
+ * page-locked host memory the device can address (swap).  `pairs` must be
+ * device-accessible (int32 [num_pairs][2]).  Out-of-range ids set
+ * PKV_FLAG_BAD_BLOCK and skip the pair.  block_bytes and scale_bytes_per_block
+ * are multiples of 16; pointers 16-byte aligned.  Source and destination
+ * blocks must not overlap.
+ */
+int pkv_copy_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                    size_t block_bytes, int dst_num_blocks, int src_num_blocks, float* dst_k_scale,
+                    float* dst_v_scale, const float* src_k_scale, const float* src_v_scale,
+                    size_t scale_bytes_per_block, const int32_t* pairs, int num_pairs,
+                    int* err_flag, pkv_stream_t stream);
 
 /* Human-readable text for a pkv_status. */
 const char* pkv_strerror(int status);

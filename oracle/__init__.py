@@ -32,6 +32,7 @@ __all__ = [
     "quantize_row_fp8",
     "append_fp8",
     "paged_decode_fp8",
+    "copy_blocks",
 ]
 
 _LIB = None
@@ -72,6 +73,8 @@ def _lib():
         lib.oracle_append_fp8.argtypes = [_vp, _vp, _i64, _i32, _i32, _vp, _vp, _i64, _i64]
         lib.oracle_paged_decode_fp8.restype = _i32
         lib.oracle_paged_decode_fp8.argtypes = [_vp] * 7 + [_i32, _vp] + [_i32] * 6 + [_dbl, _i32]
+        lib.oracle_copy_blocks.restype = _i32
+        lib.oracle_copy_blocks.argtypes = [_vp, _vp, _i64, _i32, _i32, _vp, _i32]
         lib.oracle_max_threads.restype = _i32
         lib.oracle_max_threads.argtypes = []
         _LIB = lib
@@ -249,3 +252,14 @@ def paged_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, block_tables, contex
                                         float(softmax_scale), int(threads))
     _check(rc, "oracle_paged_decode_fp8")
     return out
+
+
+def copy_blocks(dst: np.ndarray, src: np.ndarray, pairs: np.ndarray) -> None:
+    """dst[pairs[i, 1]] = src[pairs[i, 0]] for whole blocks (first axis), in place."""
+    assert dst.dtype == src.dtype and dst.shape[1:] == src.shape[1:] and dst.flags.c_contiguous
+    sb, sp = _c(src, src.dtype)
+    pb, pp = _c(pairs, np.int32)
+    block_bytes = src.dtype.itemsize * int(np.prod(src.shape[1:]))
+    rc = _lib().oracle_copy_blocks(dst.ctypes.data_as(_vp), sp, block_bytes, dst.shape[0],
+                                   src.shape[0], pp, pb.shape[0])
+    _check(rc, "oracle_copy_blocks")

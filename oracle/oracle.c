@@ -224,6 +224,20 @@ int oracle_append_int8(const float* x, const int64_t* slot_mapping, int64_t num_
   return ORACLE_OK;
 }
 
+/* Whole-block copy between pools (copy-on-write, swap): block pairs[2i] of src
+ * to block pairs[2i+1] of dst, block_bytes each.  Out-of-range ids are an error
+ * and nothing further is copied. */
+int oracle_copy_blocks(uint8_t* dst, const uint8_t* src, int64_t block_bytes, int dst_blocks,
+                       int src_blocks, const int32_t* pairs, int num_pairs) {
+  if (!dst || !src || !pairs || block_bytes <= 0 || num_pairs < 0) return ORACLE_ERR_ARG;
+  for (int i = 0; i < num_pairs; ++i) {
+    const int32_t s = pairs[2 * i], d = pairs[2 * i + 1];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) return ORACLE_ERR_BLOCK;
+    memcpy(dst + (int64_t)d * block_bytes, src + (int64_t)s * block_bytes, (size_t)block_bytes);
+  }
+  return ORACLE_OK;
+}
+
 /* ---------------------------------------------------------------- gather */
 
 /* Gather kv head kvh of sequence s's first ctx tokens into contiguous fp64

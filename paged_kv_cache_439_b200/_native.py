@@ -19,6 +19,7 @@ PKV_FLAG_CTX_RANGE = 4
 PKV_FLAG_NEG_CTX = 8
 
 PKV_ERR_SCRATCH_LIMIT = -8
+PKV_ERR_NO_BLOCKS = -9
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 # exported symbol -> (restype, argtypes); mirrors include/pkv.h
@@ -38,6 +39,22 @@ SIGNATURES = {
                                                       _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                                       _i, _vp, _sz, _i, _vp, _vp]),
     "pkv_copy": (_i, [_vp, _vp, _sz, _vp]),
+    "pkv_copy_blocks": (_i, [_vp, _vp, _vp, _vp, _sz, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp, _i,
+                             _vp, _vp]),
+    "pkv_bm_create": (_i, [_i, _i, ctypes.POINTER(ctypes.c_void_p)]),
+    "pkv_bm_destroy": (None, [_vp]),
+    "pkv_bm_num_free": (_i, [_vp]),
+    "pkv_bm_ref_count": (_i, [_vp, ctypes.c_int32]),
+    "pkv_bm_add_sequence": (_i, [_vp, ctypes.c_int64]),
+    "pkv_bm_fork": (_i, [_vp, ctypes.c_int64, ctypes.c_int64]),
+    "pkv_bm_blocks_needed": (_i, [_vp, ctypes.c_int64, _i]),
+    "pkv_bm_reserve": (_i, [_vp, ctypes.c_int64, _i, _vp, _vp, ctypes.POINTER(_i)]),
+    "pkv_bm_free": (_i, [_vp, ctypes.c_int64]),
+    "pkv_bm_seq_len": (_i, [_vp, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64),
+                            ctypes.POINTER(_i)]),
+    "pkv_bm_block_tables": (_i, [_vp, _vp, _i, _i, _vp, _vp]),
+    "pkv_bm_swap_out": (_i, [_vp, _vp, ctypes.c_int64, _vp, _i, ctypes.POINTER(_i)]),
+    "pkv_bm_swap_in": (_i, [_vp, _vp, ctypes.c_int64, _vp, _i, ctypes.POINTER(_i)]),
     "pkv_strerror": (ctypes.c_char_p, [_i]),
     "pkv_version": (_i, []),
 }

@@ -2,7 +2,8 @@
 
     python -m paged_kv_cache_439_b200.build [--force] [--verbose]
 
-Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel),
+Each ``csrc/*.cu`` (device code) and ``csrc/*.cpp`` (host code) is compiled
+to an object under ``_build/`` (in parallel),
 then linked into ``paged_kv_cache_439_b200/libpkv.so``.  Rebuilds only what is
 older than its sources or headers.
 """
@@ -47,7 +48,8 @@ def _stale(target: str, sources: list) -> bool:
 
 
 def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src).replace(".cu", ".o"))
+    base = os.path.basename(src)
+    obj = os.path.join(BUILD, base.rsplit(".", 1)[0] + (".cu.o" if base.endswith(".cu") else ".cpp.o"))
     if _stale(obj, [src] + _deps()):
         cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
         if verbose:
@@ -59,7 +61,7 @@ def _compile(src: str, verbose: bool) -> str:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
-    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     if force:
         for o in glob.glob(os.path.join(BUILD, "*.o")):
             os.remove(o)

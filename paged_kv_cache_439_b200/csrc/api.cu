@@ -140,6 +140,7 @@ const char* pkv_strerror(int status) {
     case PKV_ERR_WORKSPACE: return "workspace missing or smaller than pkv_workspace_size()";
     case PKV_ERR_CUDA: return "CUDA runtime error";
     case PKV_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case PKV_ERR_NO_BLOCKS: return "the block pool has too few free blocks";
     case PKV_ERR_SCRATCH_LIMIT:
       return "split-K scratch for this shape exceeds the fixed no-allocation scratch "
              "(PKV_NOALLOC_SCRATCH_BYTES); use pkv_paged_attention_decode with a workspace";

@@ -456,3 +456,13 @@ def test_fp8_decode_equals_attention_on_dequantised_values():
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
     plain = oracle.paged_decode(q, kf, vf, tables, cl, 0.25)
     assert np.abs(got - plain).max() < 0.2
+
+
+def test_copy_blocks_definition():
+    src = np.arange(5 * 3 * 2, dtype=np.int16).reshape(5, 3, 2)
+    dst = np.full((4, 3, 2), -1, dtype=np.int16)
+    oracle.copy_blocks(dst, src, np.array([[4, 0], [1, 3]], dtype=np.int32))
+    assert (dst[0] == src[4]).all() and (dst[3] == src[1]).all()
+    assert (dst[1] == -1).all() and (dst[2] == -1).all()
+    with pytest.raises(oracle.OracleError):
+        oracle.copy_blocks(dst, src, np.array([[5, 0]], dtype=np.int32))
