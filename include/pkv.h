@@ -64,6 +64,8 @@ typedef enum {
 #define PKV_FLAG_CTX_RANGE 4   /* context_len > max_blocks_per_seq * block_size or
                                   > max_context_len: clamped */
 #define PKV_FLAG_NEG_CTX 8     /* negative context_len: treated as 0 */
+#define PKV_FLAG_TIMEOUT 16    /* a kernel's bounded wait on its own tensor-core work gave up:
+                                  its outputs are not valid (should never be seen) */
 
 /* Supported sets: head_dim in {64, 128}; block_size a power of two in [8, 256];
  * group = num_q_heads / num_kv_heads in [1, 16]. */

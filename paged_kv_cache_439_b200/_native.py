@@ -17,6 +17,7 @@ PKV_FLAG_BAD_BLOCK = 1
 PKV_FLAG_BAD_SLOT = 2
 PKV_FLAG_CTX_RANGE = 4
 PKV_FLAG_NEG_CTX = 8
+PKV_FLAG_TIMEOUT = 16
 
 PKV_ERR_SCRATCH_LIMIT = -8
 PKV_ERR_NO_BLOCKS = -9

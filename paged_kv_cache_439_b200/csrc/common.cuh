@@ -145,6 +145,22 @@ __device__ __forceinline__ uint32_t e4m3pair_to_f16x2(uint32_t x) {
   return r;
 }
 
+// The E4M3 codes in the low (LO) or high half of x -> two exact fp16 values,
+// the lower byte in the low half of the result.
+template <bool LO>
+__device__ __forceinline__ uint32_t e4m3half_to_f16x2(uint32_t x) {
+  uint32_t r;
+  if constexpr (LO)
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, lo;\n}\n"
+        : "=r"(r)
+        : "r"(x));
+  else
+    asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n cvt.rn.f16x2.e4m3x2 %0, hi;\n}\n"
+        : "=r"(r)
+        : "r"(x));
+  return r;
+}
+
 // Two fp32 values -> two E4M3 codes (round to nearest even, saturated to
 // +-448); `lo` lands in bits 0-7.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {

@@ -218,13 +218,17 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 //
 // Tile math: scores S^T = K * Q^T and the update O^T += V^T * P^T on
 // mma.sync m16n8k16 with fp32 accumulation (16 tokens x 8 q heads per
-// instruction).  P is split into hi + lo halves so the probabilities keep ~16
-// significant bits.  INT8 codes become exact fp16 values in registers; the
-// per-token scales multiply the fp32 scores (K) and P (V).  FP8 (E4M3) codes
-// convert to exact fp16 with cvt.rn.f16x2.e4m3x2.  INT8 codes reach the
-// tensor core as the exact fp16 values code + 1152 (one byte permute per pair,
-// no subtraction); the constant is removed from the fp32 results: 1152 *
-// sum_d q[h][d] from every score, 1152 * sum_t P[t][h] from the output.
+// instruction).  For bf16 caches P is split into bf16 hi + lo halves so the
+// probabilities keep ~16 significant bits.  One-byte caches feed V as fp16, so
+// P goes in as one fp16 value (11 significant bits; its rounding error, below
+// 2^-11 of each term, is under the bf16 rounding of the output).  INT8 codes
+// become exact fp16 values in registers; the per-token scales multiply the
+// fp32 scores (K) and P (V).  FP8 (E4M3) codes convert to exact fp16 with
+// cvt.rn.f16x2.e4m3x2.  INT8 codes reach the tensor core as the exact fp16
+// values code + 1152 (one byte permute per pair, no subtraction); the constant
+// is removed from the fp32 results: 1152 * sum_d q[h][d] from every score, and
+// 1152 * sum_t P[t][h] from the output, summed over the fp16 P the tensor core
+// used so that it cancels exactly.
 
 #ifndef PKV_MMA_WARPS
 #define PKV_MMA_WARPS 4
@@ -486,10 +490,11 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       svb = __shfl_sync(0xffffffffu, mine, 24 + g);
       dep = __float_as_uint(mine);
     }
+    // one register of each ldmatrix: an ldmatrix completes all of its registers at once
 #pragma unroll
-    for (int a = 0; a < KA; ++a) dep ^= kf[a][0] ^ kf[a][1] ^ kf[a][2] ^ kf[a][3];
+    for (int a = 0; a < KA; ++a) dep ^= kf[a][0];
 #pragma unroll
-    for (int a = 0; a < VA; ++a) dep ^= vf[a][0] ^ vf[a][1] ^ vf[a][2] ^ vf[a][3];
+    for (int a = 0; a < VA; ++a) dep ^= vf[a][0];
     const uint32_t mask =
         __ballot_sync(0xffffffffu, phys_of(p, c, s_phys, tile_t0 + (lane & 15)) >= 0) & 0xFFFFu;
 
@@ -527,15 +532,16 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
       for (int kp = 0; kp < KS / 2; ++kp) {
         // kf[kp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1); bytes of a
-        // register are d 4t..4t+3 -> slots (2t, 2t+1) and (2t+8, 2t+9)
+        // register are d 4t..4t+3 -> slots (2t, 2t+1) (its low half) and
+        // (2t+8, 2t+9) (its high half), so each half converts as it is
         const uint32_t top[2] = {kf[kp][0], kf[kp][2]};
         const uint32_t bot[2] = {kf[kp][1], kf[kp][3]};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = e4m3pair_to_f16x2<0x0010>(top[h]);
-          const uint32_t a2 = e4m3pair_to_f16x2<0x0032>(top[h]);
-          const uint32_t a1 = e4m3pair_to_f16x2<0x0010>(bot[h]);
-          const uint32_t a3 = e4m3pair_to_f16x2<0x0032>(bot[h]);
+          const uint32_t a0 = e4m3half_to_f16x2<true>(top[h]);
+          const uint32_t a2 = e4m3half_to_f16x2<false>(top[h]);
+          const uint32_t a1 = e4m3half_to_f16x2<true>(bot[h]);
+          const uint32_t a3 = e4m3half_to_f16x2<false>(bot[h]);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             if (h)
@@ -606,28 +612,23 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         rescale |= (a != 1.f);
       }
       const float q0 = pr[0] * pva, q1 = pr[1] * pva, q2 = pr[2] * pvb, q3 = pr[3] * pvb;
-      if constexpr (I8) {
-        p_run[nt][0] = p_run[nt][0] * alpha[nt][0] + (q0 + q2);
-        p_run[nt][1] = p_run[nt][1] * alpha[nt][1] + (q1 + q3);
-      }
-      uint32_t h01, h23, l01, l23;
       if constexpr (!Q8) {
-        h01 = pack_bf16(q0, q1);
-        h23 = pack_bf16(q2, q3);
+        const uint32_t h01 = pack_bf16(q0, q1), h23 = pack_bf16(q2, q3);
         const float2 f01 = unpack_bf16(h01), f23 = unpack_bf16(h23);
-        l01 = pack_bf16(q0 - f01.x, q1 - f01.y);
-        l23 = pack_bf16(q2 - f23.x, q3 - f23.y);
+        bh[nt][0] = movmatrix_trans(h01);
+        bh[nt][1] = movmatrix_trans(h23);
+        bl[nt][0] = movmatrix_trans(pack_bf16(q0 - f01.x, q1 - f01.y));
+        bl[nt][1] = movmatrix_trans(pack_bf16(q2 - f23.x, q3 - f23.y));
       } else {
-        h01 = pack_f16(q0, q1);
-        h23 = pack_f16(q2, q3);
-        const float2 f01 = unpack_f16(h01), f23 = unpack_f16(h23);
-        l01 = pack_f16(q0 - f01.x, q1 - f01.y);
-        l23 = pack_f16(q2 - f23.x, q3 - f23.y);
+        const uint32_t h01 = pack_f16(q0, q1), h23 = pack_f16(q2, q3);
+        if constexpr (I8) {  // the P the tensor core sees, for the 1152 bias
+          const float2 f01 = unpack_f16(h01), f23 = unpack_f16(h23);
+          p_run[nt][0] = p_run[nt][0] * alpha[nt][0] + (f01.x + f23.x);
+          p_run[nt][1] = p_run[nt][1] * alpha[nt][1] + (f01.y + f23.y);
+        }
+        bh[nt][0] = movmatrix_trans(h01);
+        bh[nt][1] = movmatrix_trans(h23);
       }
-      bh[nt][0] = movmatrix_trans(h01);
-      bh[nt][1] = movmatrix_trans(h23);
-      bl[nt][0] = movmatrix_trans(l01);
-      bl[nt][1] = movmatrix_trans(l23);
     }
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -667,7 +668,6 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
           }
         }
       }
@@ -687,7 +687,6 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
           }
         }
       }
@@ -924,15 +923,17 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 // ---------------------------------------------------------------------------
 // Split merge: out = sum_k 2^{lse_k} o_k / sum_k 2^{lse_k} over the partials
 // of one (sequence, q head): the shared-prefix slots [0, ws_base) and the
-// splits that hold tokens.  One warp per (q head, sequence): the lanes first
-// turn the log2-sum-exps into weights (in shared memory), then each lane sums
-// four head_dim columns of the weighted partials with 16-byte loads.
+// splits that hold tokens (every one of them was written, so all are finite).
+// One warp per (q head, sequence); lane l sums head_dim columns 4l..4l+3 of the
+// weighted partials with 16-byte loads.  The first kMergeBatch partial rows are
+// loaded before the weights are known, so their latency overlaps the
+// log-sum-exp reads; the weights are held one per lane and broadcast with
+// shuffles, 32 slots per round.
 constexpr int kMergeWarps = 4;
-constexpr int kMergeMaxSlots = 256;  // slots per warp held in shared memory at once
+constexpr int kMergeBatch = 8;  // partial rows in flight per lane
 
 template <int HD>
 __global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeParams p) {
-  __shared__ float s_w[kMergeWarps][kMergeMaxSlots];
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int qh = blockIdx.x * kMergeWarps + warp, seq = blockIdx.y;
   if (qh >= p.num_q_heads) return;
@@ -940,41 +941,50 @@ __global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeP
   const int rest = ctx > p.t_start ? ctx - p.t_start : 0;
   const int n = p.ws_base + (rest + p.chunk - 1) / p.chunk;
   const size_t r = ((size_t)seq * p.num_q_heads + qh) * p.ws_slots;
-  float* w = s_w[warp];
+  const bool cols = lane * 4 < HD;
+  const float4* src = reinterpret_cast<const float4*>(p.ws_o + r * HD) + lane;
+  constexpr int kRow = HD / 4;  // float4 per partial row
+
+  float4 v[kMergeBatch];
+#pragma unroll
+  for (int i = 0; i < kMergeBatch; ++i)
+    if (cols && i < n) v[i] = src[(size_t)i * kRow];
+  float M = -CUDART_INF_F;
+  for (int k = lane; k < n; k += kWarp) M = fmaxf(M, p.ws_lse[r + k]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float L = 0.f;
-  // slots in rounds of kMergeMaxSlots (one round unless the plan is huge)
-  for (int base = 0; base < n; base += kMergeMaxSlots) {
-    const int cnt = min(n - base, kMergeMaxSlots);
-    float M = -CUDART_INF_F;
-    for (int k = lane; k < n; k += kWarp) M = fmaxf(M, p.ws_lse[r + k]);
+  if (M != -CUDART_INF_F) {
+    for (int base = 0; base < n; base += kWarp) {
+      const int cnt = min(n - base, kWarp);
+      const float lse = lane < cnt ? p.ws_lse[r + base + lane] : -CUDART_INF_F;
+      const float w = lse == -CUDART_INF_F ? 0.f : exp2f(lse - M);
+      float ws = w;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    if (M == -CUDART_INF_F) break;
-    for (int k = lane; k < cnt; k += kWarp) {
-      const float lse = p.ws_lse[r + base + k];
-      w[k] = lse == -CUDART_INF_F ? 0.f : exp2f(lse - M);
-    }
-    __syncwarp();
-    if (base == 0) L = 0.f;
-    // weights relative to the max over all slots, so rounds add up directly
-    for (int k = 0; k < cnt; ++k) L += w[k];
-    if (lane * 4 < HD) {
-#pragma unroll 4
-      for (int k = 0; k < cnt; ++k) {
-        const float wk = w[k];
-        if (wk == 0.f) continue;
-        const float4 v =
-            *reinterpret_cast<const float4*>(p.ws_o + (r + base + k) * HD + lane * 4);
-        acc[0] += wk * v.x;
-        acc[1] += wk * v.y;
-        acc[2] += wk * v.z;
-        acc[3] += wk * v.w;
+      for (int off = 16; off > 0; off >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, off);
+      L += ws;
+      for (int k0 = 0; k0 < cnt; k0 += kMergeBatch) {
+        if (base + k0 >= kMergeBatch) {  // the first batch is already in registers
+#pragma unroll
+          for (int i = 0; i < kMergeBatch; ++i)
+            if (cols && k0 + i < cnt) v[i] = src[(size_t)(base + k0 + i) * kRow];
+        }
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+          const float wk = __shfl_sync(0xffffffffu, w, (k0 + i) & (kWarp - 1));
+          if (k0 + i < cnt) {
+            acc[0] += wk * v[i].x;
+            acc[1] += wk * v[i].y;
+            acc[2] += wk * v[i].z;
+            acc[3] += wk * v[i].w;
+          }
+        }
       }
     }
-    __syncwarp();
   }
-  if (lane * 4 >= HD) return;
+  if (!cols) return;
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const size_t o = ((size_t)seq * p.num_q_heads + qh) * HD + lane * 4;
   if (p.out_f32) {

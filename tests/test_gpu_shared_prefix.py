@@ -89,3 +89,33 @@ def test_full_shared_prefix_workload(bs):
     r = assert_close(out, ref, tol_for(wl), f"shared-prefix bs={bs}")
     assert g.flags() == 0
     print(f"shared-prefix cascade bs={bs}: max_abs={r['max_abs']:.2e}")
+
+
+def test_ragged_prefix_tiles():
+    # prefix of 40 tokens (5 blocks of 8): the shared slice ends inside a tile
+    lens = [40 + x for x in (1, 9, 33, 70)]
+    wl = make_custom("sp-ragged", lens, 8, 2, 128, 8, "bf16", seed=35, shared_prefix=40)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 2):
+        assert_close(_cascade(g, wl, 40, num_splits=splits), ref, tol_for(wl), "ragged")
+    assert g.flags() == 0
+
+
+def test_running_max_moves_inside_the_prefix():
+    """Keys of two later prefix blocks are scaled up so that, for many rows, a
+    later tile's scores exceed everything before by far more than 2^8 in the
+    exponent: the kernel must move its reference maximum and rescale O."""
+    prefix, bs = 512, 16
+    lens = [prefix + x for x in (3, 40, 77, 120, 1, 64, 200, 9)]
+    wl = make_custom("sp-move", lens, 16, 2, 128, bs, "bf16", seed=36, shared_prefix=prefix)
+    prefix_blocks = wl.block_tables[0, :prefix // bs]
+    blk = wl.prefill_slots // bs
+    for which, factor in ((5, 6.0), (20, 12.0)):   # tiles 1 and 5 of the prefix
+        rows = (blk == prefix_blocks[which]).nonzero().flatten()
+        wl.prefill_k[rows] = (wl.prefill_k[rows].float() * factor).to(wl.prefill_k.dtype)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1):
+        assert_close(_cascade(g, wl, prefix, num_splits=splits), ref, tol_for(wl), "moving max")
+    assert g.flags() == 0
