@@ -501,26 +501,31 @@ def main():
     except Exception:
         pass
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: the step's
+    # inputs are packed into one pinned staging buffer (16-byte aligned pieces)
+    # and moved with one host-to-device copy; the output comes back with one
+    # device-to-host copy
     e2e = None
     if not args.no_e2e:
-        hq = wl.q.pin_memory()
-        hk, hv, hs = wl.new_k.pin_memory(), wl.new_v.pin_memory(), wl.new_slots.pin_memory()
-        hbt, hcl = wl.block_tables.pin_memory(), wl.context_lens.pin_memory()
+        pieces = [wl.q, wl.new_k, wl.new_v, wl.new_slots, wl.block_tables, wl.context_lens]
+        offs, total = [], 0
+        for x in pieces:
+            offs.append(total)
+            total += (x.numel() * x.element_size() + 15) // 16 * 16
+        hbuf = torch.empty(total, dtype=torch.uint8).pin_memory()
+        dbuf = torch.empty(total, dtype=torch.uint8, device=dev)
+        views = []
+        for x, o in zip(pieces, offs):
+            n = x.numel() * x.element_size()
+            hbuf[o:o + n].copy_(x.contiguous().view(-1).view(torch.uint8))
+            views.append(dbuf[o:o + n].view(x.dtype).view(x.shape))
+        dq, dk, dv, dsl, dbt, dcl = views
         hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hs, hbt, hcl))
+        h2d = sum(x.numel() * x.element_size() for x in pieces)
         d2h = hout.numel() * hout.element_size()
-        dq, dk, dv, dsl = torch.empty_like(q), torch.empty_like(nk), torch.empty_like(nv), \
-            torch.empty_like(ns)
-        dbt, dcl = torch.empty_like(bt), torch.empty_like(cl)
 
         def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            dsl.copy_(hs, non_blocking=True)
-            dbt.copy_(hbt, non_blocking=True)
-            dcl.copy_(hcl, non_blocking=True)
+            dbuf.copy_(hbuf, non_blocking=True)
             pkv.kv_cache_append(dk, dv, dsl, k_cache, v_cache, k_scale, v_scale, err_flag=err)
             attend(dq, dbt, dcl)
             hout.copy_(out, non_blocking=True)

@@ -103,8 +103,7 @@ struct PrefixPlan {
 PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                        int max_ctx, int prefix_len, pkv_dtype cache_dt, int num_splits) {
   PrefixPlan pl;
-  const long long rows = (long long)num_seqs * (num_q_heads / num_kv_heads);
-  const long long rg = (rows + pkv::prefix_rows_per_cta() - 1) / pkv::prefix_rows_per_cta();
+  const long long rg = pkv::prefix_row_groups(num_seqs, num_q_heads / num_kv_heads);
   const long long target = 2LL * sm_count();
   long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
   const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;

@@ -51,7 +51,8 @@ cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_di
                           cudaStream_t st);
 cudaError_t launch_prefix(const DecodeParams& p, const PrefixParams& pp, int head_dim,
                           cudaStream_t st);
-int prefix_rows_per_cta();
+// CTAs of rows per KV head in the shared-prefix pass (128 / group sequences each).
+int prefix_row_groups(int num_seqs, int group);
 cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st);
 int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim);
 

@@ -13,8 +13,9 @@
 // workspace.  The per-sequence suffix runs through the split decode kernel
 // from token prefix_len on, and the merge kernel combines both exactly.
 //
-// The rows of one KV head form a dense contraction, so one CTA takes 128 rows
-// (the M of one tcgen05.mma) and walks its slice in 64-token tiles:
+// The rows of one KV head form a dense contraction, so one CTA takes 128 / group
+// whole sequences, up to 128 rows (the M of one tcgen05.mma), and walks its
+// slice in 64-token tiles:
 //   S = Q K^T      tcgen05.mma, A = Q and B = K from shared memory (K-major,
 //                  128-byte swizzle), D = S in tensor memory (128 lanes x 64
 //                  fp32 columns);
@@ -26,16 +27,24 @@
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 2^8 (then O is rescaled in tensor memory): exponentials stay below 256,
 // and the final normalisation uses the same maximum as every P, so the result
-// is the same softmax.  One thread issues the MMAs; tcgen05.commit arrives on
-// an mbarrier the other threads wait on, each wait bounded.  K and V tiles are
-// gathered from the paged blocks with cp.async into two-stage rings of their
-// own: K tile j + 2 is fetched as soon as S of tile j is in tensor memory, V
-// tile j + 1 as soon as P V of tile j - 1 is done, so every copy has a whole
-// tile of work to land behind.  Two CTAs share an SM (half of its tensor
-// memory each), so one CTA's softmax overlaps the other's MMAs.
+// is the same softmax.  One thread issues the copies and the MMAs; copies and
+// tcgen05.commit arrive on mbarriers, each wait bounded.  Q, K and V move by
+// TMA (cp.async.bulk.tensor) straight into the 128-byte-swizzled layout the
+// MMAs read: Q as a (sequences x heads x 64 columns) box, the K and V tiles
+// as one box per paged block (or 64-token piece of one) and column block, a
+// bad block being read from past the end of the cache (zero fill).  K and V
+// have two-stage rings of their own: K tile j + 2 is fetched as soon as S of
+// tile j is in tensor memory, V tile j + 1 once P V of tile j - 1 is done.  Two
+// CTAs share an SM (half of its tensor memory each), so one CTA's softmax
+// overlaps the other's MMAs.  The softmax keeps eight independent max and
+// sum chains per row.
 #include <math_constants.h>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <atomic>
+#include <mutex>
 
 #include "common.cuh"
 #include "decode.cuh"
@@ -71,12 +80,6 @@ struct TcCfg {
   static constexpr int BODY = Q_BYTES + 2 * kTcStages * KV_BYTES;
   static_assert(HD == 64 || HD == 128, "head_dim 64 or 128");
 };
-
-// 128-byte swizzle: 16-byte chunk c of the 128-byte row r of a 1024-byte
-// aligned atom lives at chunk c ^ (r & 7).
-__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
 // stride byte offsets (all >> 4), version 1, 128-byte swizzle.
@@ -148,8 +151,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     if (done) return true;
     if (i == 0) t0 = global_ns();
-    else if ((i & 63) == 0 && global_ns() - t0 > kWaitNs) return false;
+    else if ((i & 15) == 0 && global_ns() - t0 > kWaitNs) return false;
+    __nanosleep(32);
   }
+}
+
+// One lane per warp polls while the others wait at the warp barrier, so that
+// waiting warps do not flood the shared-memory pipe that the copies and the
+// tensor-memory loads go through.  Every lane gets the verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
 }
 
 // 32 consecutive fp32 columns of this thread's tensor-memory lane.
@@ -189,9 +204,44 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Arrives on `bar` (count 1) and adds `bytes` of expected copy transactions.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+// Adds `bytes` of expected copy transactions without arriving.
+__device__ __forceinline__ void mbar_add_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// One box of a 3-D tensor map into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// Max of 64 values in 8 independent chains.
+__device__ __forceinline__ float max64(const float (&v)[kTcTok]) {
+  float m[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m[c] = v[c];
+#pragma unroll
+  for (int i = 8; i < kTcTok; i += 8)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) m[c] = fmaxf(m[c], v[i + c]);
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
 template <int HD>
-__global__ void __launch_bounds__(kTcThreads)
-    prefix_kernel(const DecodeParams p, const PrefixParams pp) {
+__global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
+    prefix_kernel(const DecodeParams p, const PrefixParams pp,
+                  const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v) {
   using Cfg = TcCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -204,15 +254,19 @@ __global__ void __launch_bounds__(kTcThreads)
   uint8_t* const tail = gbase + Cfg::BODY + pp.phys_bytes;
   const uint32_t bar_s = smem_u32(tail);       // S of a tile is in tensor memory
   const uint32_t bar_o = smem_u32(tail + 8);   // a tile's P V has been accumulated
-  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 16);
+  const uint32_t bar_k = smem_u32(tail + 16);  // [2]: K tile (and, first, Q) landed
+  const uint32_t bar_v = smem_u32(tail + 32);  // [2]: V tile landed
+  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 48);
 
   const int kvh = blockIdx.x, split = blockIdx.y, rg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / kWarp;
   const int G = p.group;
+  const int spc = kTcRows / G;  // sequences per CTA; rows (seq, head) = spc * G <= 128
   const int t0 = split * pp.pchunk;
   const int t1 = min(pp.prefix_len, t0 + pp.pchunk);
   const int bs = p.block_size;
   const int blk0 = t0 >> p.log2_bs;
+  const int ntiles = (t1 - t0 + kTcTok - 1) / kTcTok;
 
   // ---- set-up: block-table slice, barriers, tensor memory
   {
@@ -229,6 +283,10 @@ __global__ void __launch_bounds__(kTcThreads)
   if (tid == 0) {
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_k + 8, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_v + 8, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -238,13 +296,19 @@ __global__ void __launch_bounds__(kTcThreads)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // Q rows past spc * G (when G does not divide 128) are never loaded: zero them
+  for (int rr = spc * G + tid / 8; rr < kTcRows; rr += kTcThreads / 8)
+#pragma unroll
+    for (int db = 0; db < Cfg::DB; ++db)
+      *reinterpret_cast<uint4*>(gbase + db * Cfg::Q_DB + rr * 128 + (tid % 8) * 16) =
+          make_uint4(0, 0, 0, 0);
+  fence_async_smem();
 
   // ---- this thread's row
   const int row = tid;
-  const int r = rg * kTcRows + row;
-  const bool rvalid = r < pp.rows;
-  const int seq = rvalid ? r / G : 0;
-  const size_t qrow = (size_t)seq * p.num_q_heads + kvh * G + (rvalid ? r % G : 0);
+  const int seq = rg * spc + row / G;
+  const bool rvalid = row < spc * G && seq < p.num_seqs;
+  const size_t qrow = (size_t)(rvalid ? seq : 0) * p.num_q_heads + kvh * G + row % G;
   int lim = 0;  // tokens of the prefix this row attends to
   if (rvalid) {
     int ctx = p.context_lens[seq];
@@ -252,58 +316,28 @@ __global__ void __launch_bounds__(kTcThreads)
     lim = min(ctx, pp.prefix_len);
   }
 
-  // ---- copies: Q (once) and the K/V tiles, into the swizzled column blocks
-  const uint8_t* kb = static_cast<const uint8_t*>(p.k_cache);
-  const uint8_t* vb = static_cast<const uint8_t*>(p.v_cache);
-  const size_t tok_stride = (size_t)p.num_kv_heads * HD * 2;
-  __syncthreads();  // s_phys
-  {
-    const uint8_t* qb = static_cast<const uint8_t*>(p.q);
-    constexpr int CH = HD / 8;  // 16-byte chunks per row
-#pragma unroll 4
-    for (int i = tid; i < kTcRows * CH; i += kTcThreads) {
-      const int rr = i / CH, c = i % CH;
-      const int gr = rg * kTcRows + rr;
-      const bool ok = gr < pp.rows;
-      const size_t qr = ok ? (size_t)(gr / G) * p.num_q_heads + kvh * G + gr % G : 0;
-      cp_async_16(q_sm + (uint32_t)((c >> 3) * Cfg::Q_DB) + sw128(rr, c & 7),
-                  qb + qr * HD * 2 + (size_t)c * 16, ok ? 16 : 0);
-    }
-  }
-  const int ntiles = (t1 - t0 + kTcTok - 1) / kTcTok;
-  // copies of K (or V) tile j into its ring stage; rows past the slice or in a
-  // bad block are zero-filled
-  auto copy_tile = [&](const uint8_t* src, uint32_t ring_base, int j) {
-    constexpr int CH = HD / 8;
+  // ---- tile copies (thread 0): K or V tile j as boxes of R token rows x 64
+  // head_dim columns, one per (block piece, column block); a bad block, or
+  // rows past the slice, load from past the end of the cache: zeros
+  const int R = bs < kTcTok ? bs : kTcTok;
+  const int oob = p.num_blocks * bs;
+  auto load_tile = [&](const CUtensorMap* map, uint32_t stage, int j, uint32_t bar) {
+    mbar_expect_tx(bar, Cfg::KV_BYTES);
     const int tt = t0 + j * kTcTok;
-    const uint32_t st = ring_base + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES);
-#pragma unroll 4
-    for (int i = tid; i < kTcTok * CH; i += kTcThreads) {
-      const int rr = i / CH, c = i % CH;
-      const int t = tt + rr;
+    for (int b = 0; b < kTcTok / R; ++b) {
+      const int t = tt + b * R;
       const int phys = t < t1 ? s_phys[(t >> p.log2_bs) - blk0] : -1;
-      size_t off = 0;
-      int n = 0;
-      if (phys >= 0) {
-        off = ((size_t)phys * bs + (t & (bs - 1))) * tok_stride + (size_t)kvh * HD * 2 +
-              (size_t)c * 16;
-        n = 16;
-      }
-      cp_async_16(st + (uint32_t)((c >> 3) * Cfg::KV_DB) + sw128(rr, c & 7), src + off, n);
+      const int z = phys >= 0 ? phys * bs + (t & (bs - 1)) : oob;
+#pragma unroll
+      for (int db = 0; db < Cfg::DB; ++db)
+        tma_load_3d(stage + (uint32_t)(db * Cfg::KV_DB + b * R * 128), map, db * 64, kvh, z, bar);
     }
   };
-  // one commit group per call (empty past the last tile, to keep the count)
-  auto issue_tile = [&](const uint8_t* src, uint32_t ring_base, int j) {
-    if (j < ntiles) copy_tile(src, ring_base, j);
-    cp_async_commit();
-  };
-  // groups in commit order: {Q, V0, K0}, {K1}, then per tile j: {K j+2}, {V j+1}
-  copy_tile(vb, v_ring, 0);
-  issue_tile(kb, k_ring, 0);
-  issue_tile(kb, k_ring, 1);
+  auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
+  auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
 
   tc_fence_before();
-  __syncthreads();  // barriers initialised, tensor-memory address written
+  __syncthreads();  // s_phys, barriers, tensor-memory address, zeroed Q rows
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
@@ -311,7 +345,7 @@ __global__ void __launch_bounds__(kTcThreads)
   constexpr uint32_t kIdQK = idesc_bf16(kTcRows, kTcTok, 0);
   constexpr uint32_t kIdPV = idesc_bf16(kTcRows, HD, 1);
   auto issue_qk = [&](int j) {  // S = Q K^T of tile j (thread 0)
-    const uint32_t kS = k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES);
+    const uint32_t kS = kstage(j);
 #pragma unroll
     for (int ks = 0; ks < HD / 16; ++ks) {
       const uint32_t koff = (uint32_t)((ks >> 2) * Cfg::KV_DB + (ks & 3) * 32);
@@ -322,7 +356,7 @@ __global__ void __launch_bounds__(kTcThreads)
     mma_commit(bar_s);
   };
   auto issue_pv = [&](int j) {  // O += P V of tile j (thread 0)
-    const uint32_t vS = v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES);
+    const uint32_t vS = vstage(j);
 #pragma unroll
     for (int kk = 0; kk < kTcTok / 16; ++kk) {
       const uint64_t bd = smem_desc(vS + (uint32_t)(kk * 16 * 128), Cfg::KV_DB, 1024);
@@ -332,24 +366,34 @@ __global__ void __launch_bounds__(kTcThreads)
     mma_commit(bar_o);
   };
 
-  // first tile: data (and Q) landed -> visible to the tensor cores -> S_0
-  cp_async_wait<1>();
-  fence_async_smem();
-  __syncthreads();
+  // ---- prologue (thread 0): Q with K0, V0, K1, V1; then S of tile 0
+  bool ok = true;
   if (tid == 0) {
+    mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
+#pragma unroll
+    for (int db = 0; db < Cfg::DB; ++db)
+      tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
+    load_tile(&tm_k, kstage(0), 0, bar_k);
+    load_tile(&tm_v, vstage(0), 0, bar_v);
+    if (ntiles > 1) {
+      load_tile(&tm_k, kstage(1), 1, bar_k + 8);
+      load_tile(&tm_v, vstage(1), 1, bar_v + 8);
+    }
+    ok = mbar_wait(bar_k, 0);
     tc_fence_after();
-    issue_qk(0);
+    if (ok) issue_qk(0);
   }
 
-  float m_ref = -CUDART_INF_F;  // reference maximum of this row (log2 units)
+  float m_ref = -CUDART_INF_F;  // reference maximum of this row (scaled, log2 units)
   float l_run = 0.f;
   bool failed = false;
+  const float sc = p.scale_log2;
   for (int j = 0; j < ntiles; ++j) {
     const int tt = t0 + j * kTcTok;
-    // ---- scores of tile j
-    bool ok = mbar_wait(bar_s, (uint32_t)(j & 1));
+    // ---- scores of tile j; its K stage takes tile j + 2
+    ok &= warp_wait(bar_s, (uint32_t)(j & 1));
     tc_fence_after();
-    issue_tile(kb, k_ring, j + 2);  // K tile j has been consumed
+    if (tid == 0 && j + 2 < ntiles) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
     float s[kTcTok];
     {
       float a[32], b[32];
@@ -368,14 +412,18 @@ __global__ void __launch_bounds__(kTcThreads)
     for (int b = (tt >> p.log2_bs) - blk0; b <= ((min(tt + kTcTok, t1) - 1) >> p.log2_bs) - blk0;
          ++b)
       bad |= s_phys[b] < 0;
-    float mt = -CUDART_INF_F;
+    if (nval < kTcTok || bad || sc <= 0.f) {  // masked tile (or an unusual scale): the slow path
 #pragma unroll
-    for (int i = 0; i < kTcTok; ++i) {
-      bool v = i < nval;
-      if (bad) v = v && s_phys[((tt + i) >> p.log2_bs) - blk0] >= 0;
-      s[i] = v ? s[i] * p.scale_log2 : -CUDART_INF_F;
-      mt = fmaxf(mt, s[i]);
+      for (int i = 0; i < kTcTok; ++i) {
+        bool v = i < nval;
+        if (bad) v = v && s_phys[((tt + i) >> p.log2_bs) - blk0] >= 0;
+        s[i] = v ? s[i] * sc : -CUDART_INF_F;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kTcTok; ++i) s[i] *= sc;
     }
+    const float mt = max64(s);
     const bool move = mt > m_ref + kRescaleLog2;  // also true for the first valid tile
     const float m_new = move ? mt : m_ref;
     const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
@@ -383,10 +431,10 @@ __global__ void __launch_bounds__(kTcThreads)
     // ---- the previous tile's P V must be done: P is overwritten, O may be
     // rescaled, and its V stage takes tile j + 1
     if (j > 0) {
-      ok &= mbar_wait(bar_o, (uint32_t)((j - 1) & 1));
+      ok &= warp_wait(bar_o, (uint32_t)((j - 1) & 1));
       tc_fence_after();
+      if (tid == 0 && j + 1 < ntiles) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
     }
-    issue_tile(vb, v_ring, j + 1);
     // rare: rescale O in place.  tcgen05.ld/st are warp-collective, so the whole
     // warp takes this path when any of its rows needs it (alpha = 1 for the rest).
     const bool need = move && j > 0 && m_ref != -CUDART_INF_F;
@@ -408,61 +456,75 @@ __global__ void __launch_bounds__(kTcThreads)
     m_ref = m_new;
     const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
 
-    // ---- P = 2^(s - m) as bf16 hi + lo, into tensor memory
+    // ---- P = 2^(s - m) as bf16 hi + lo, into tensor memory (8 partial sums)
     {
       uint32_t hi[32], lo[32];
-      float rs = 0.f;
+      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float x0 = fast_exp2(s[2 * i] - m_use), x1 = fast_exp2(s[2 * i + 1] - m_use);
-        rs += x0 + x1;
+        rs[i & 7] += x0 + x1;
         const uint32_t h = pack_bf16(x0, x1);
         const float2 f = unpack_bf16(h);
         hi[i] = h;
         lo[i] = pack_bf16(x0 - f.x, x1 - f.y);
       }
-      l_run += rs;
+      l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       tmem_st32(tmem + lane_base + Cfg::PH_COL, hi);
       tmem_st32(tmem + lane_base + Cfg::PL_COL, lo);
       tmem_wait_st();
     }
-    // ---- V tile j and K tile j + 1 landed (the two groups of this tile may still fly)
-    cp_async_wait<2>();
-    fence_async_smem();
     tc_fence_before();
     failed = __syncthreads_or(!ok);
     if (failed) break;
-    if (tid == 0) {
+    if (tid == 0) {  // V tile j and K tile j + 1 landed -> P V of tile j, S of tile j + 1
+      ok &= mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
       tc_fence_after();
-      issue_pv(j);
-      if (j + 1 < ntiles) issue_qk(j + 1);
+      if (ok) issue_pv(j);
+      if (ok && j + 1 < ntiles) {
+        ok &= mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
+        if (ok) issue_qk(j + 1);
+      }
     }
   }
 
-  // ---- the last P V, then normalise and write this slice's partial
+  // ---- the last P V, then normalise this slice's partial.  Thread r holds
+  // row r; the rows go through shared memory (the K/V rings, now idle) so that
+  // each warp writes whole rows of the workspace.
   if (!failed) {
-    const bool ok = mbar_wait(bar_o, (uint32_t)((ntiles - 1) & 1));
+    ok &= warp_wait(bar_o, (uint32_t)((ntiles - 1) & 1));
     tc_fence_after();
-    failed = !ok;
-    const size_t slot = qrow * p.ws_slots + split;
+    failed = __syncthreads_or(!ok);
+  }
+  if (!failed) {
+    constexpr int CHK = HD / 4;  // 16-byte chunks per row
+    float4* stage = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES);
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < HD; c += 32) {
       float o[32];
       tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o);
       tmem_wait_ld();
-      if (rvalid && ok) {
-        float4* dst = reinterpret_cast<float4*>(p.ws_o + slot * HD + c);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv,
-                               o[4 * i + 3] * inv);
+      for (int i = 0; i < 8; ++i) {
+        const int ch = c / 4 + i;
+        stage[row * CHK + (ch ^ (row & (CHK - 1)))] =
+            make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
       }
     }
-    if (rvalid && ok)
-      p.ws_lse[slot] = l_run > 0.f ? m_ref + log2f(l_run) : -CUDART_INF_F;
+    if (rvalid)
+      p.ws_lse[qrow * p.ws_slots + split] = l_run > 0.f ? m_ref + log2f(l_run) : -CUDART_INF_F;
+    __syncthreads();
+    constexpr int RPI = 32 / CHK;  // rows per warp store
+    const int lane = tid & 31;
+    for (int rr = warp * RPI + lane / CHK; rr < kTcRows; rr += 4 * RPI) {
+      const int sq = rg * spc + rr / G;
+      if (rr >= spc * G || sq >= p.num_seqs) continue;
+      const size_t slot = ((size_t)sq * p.num_q_heads + kvh * G + rr % G) * p.ws_slots + split;
+      const int ch = lane % CHK;
+      reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] = stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
+    }
   }
-  cp_async_wait<0>();
   tc_fence_before();
   failed = __syncthreads_or(failed);
   if (failed && tid == 0) set_flag(p.err_flag, PKV_FLAG_TIMEOUT);
@@ -474,9 +536,42 @@ __global__ void __launch_bounds__(kTcThreads)
   }
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor [d2][d1][d0] (d0 innermost, contiguous rows) with 128-byte
+// swizzled boxes of 64 x b1 x b2 elements.
+cudaError_t bf16_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint32_t b1, uint32_t b2) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {64u, b1, b2};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int HD>
 int smem_bytes(const PrefixParams& pp) {
-  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 32;
+  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 64;
 }
 
 template <int HD>
@@ -497,14 +592,28 @@ cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, cudaStream_t s
     if (e != cudaSuccess) return e;
     ready.fetch_or(bit);
   }
-  const dim3 grid(p.num_kv_heads, pp.prefix_splits, (pp.rows + kTcRows - 1) / kTcRows);
-  k<<<grid, kTcThreads, smem, st>>>(p, pp);
+  const int G = p.group;
+  const int spc = kTcRows / G;
+  const int rows_box = p.block_size < kTcTok ? p.block_size : kTcTok;
+  const uint64_t cache_rows = (uint64_t)p.num_blocks * p.block_size;
+  CUtensorMap tq, tk, tv;
+  e = bf16_map(&tq, p.q, HD, p.num_q_heads, p.num_seqs, (uint32_t)G, (uint32_t)spc);
+  if (e == cudaSuccess)
+    e = bf16_map(&tk, p.k_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
+  if (e == cudaSuccess)
+    e = bf16_map(&tv, p.v_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(p.num_kv_heads, pp.prefix_splits, (p.num_seqs + spc - 1) / spc);
+  k<<<grid, kTcThreads, smem, st>>>(p, pp, tq, tk, tv);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int prefix_rows_per_cta() { return kTcRows; }
+int prefix_row_groups(int num_seqs, int group) {
+  const int spc = kTcRows / group;
+  return (num_seqs + spc - 1) / spc;
+}
 
 cudaError_t launch_prefix(const DecodeParams& p, const PrefixParams& pp, int head_dim,
                           cudaStream_t st) {
