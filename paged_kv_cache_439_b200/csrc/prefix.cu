@@ -27,16 +27,19 @@
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 2^8 (then O is rescaled in tensor memory): exponentials stay below 256,
 // and the final normalisation uses the same maximum as every P, so the result
-// is the same softmax.  One thread issues the copies and the MMAs; copies and
-// tcgen05.commit arrive on mbarriers, each wait bounded.  Q, K and V move by
+// is the same softmax.  A fifth warp is the producer: one of its lanes issues
+// every copy and MMA; copies, tcgen05.commit and the softmax warps' hand-offs
+// (S read, P written) arrive on mbarriers, each wait bounded.  Q, K and V move by
 // TMA (cp.async.bulk.tensor) straight into the 128-byte-swizzled layout the
 // MMAs read: Q as a (sequences x heads x 64 columns) box, the K and V tiles
 // as one box per paged block (or 64-token piece of one) and column block, a
 // bad block being read from past the end of the cache (zero fill).  K and V
-// have two-stage rings of their own: K tile j + 2 is fetched as soon as S of
-// tile j is in tensor memory, V tile j + 1 once P V of tile j - 1 is done.  Two
-// CTAs share an SM (half of its tensor memory each), so one CTA's softmax
-// overlaps the other's MMAs.  The softmax keeps eight independent max and
+// have two-stage rings of their own.  Once every row has read S of tile j
+// into registers, S of tile j + 1 is issued (it runs during tile j's softmax)
+// and K tile j + 2 is fetched; V tile j + 1 is fetched once P V of tile j - 1
+// is done.  Two CTAs share an SM (half of its tensor memory each, at most 168
+// registers a thread so that both fit), so one CTA's softmax overlaps the
+// other's MMAs.  The softmax keeps eight independent max and
 // sum chains per row.
 #include <math_constants.h>
 
@@ -53,7 +56,8 @@ namespace pkv {
 
 namespace {
 
-constexpr int kTcThreads = 128;  // one thread per row; warp w reads TMEM lanes 32w..32w+31
+constexpr int kTcSoftmaxWarps = 4;  // thread r owns row r; warp w reads TMEM lanes 32w..32w+31
+constexpr int kTcThreads = (kTcSoftmaxWarps + 1) * 32;  // plus one producer warp
 constexpr int kTcRows = 128;     // rows per CTA (MMA M)
 constexpr int kTcTok = kPrefixTokens;  // tokens per tile (MMA N of Q K^T)
 constexpr int kTcStages = 2;
@@ -152,7 +156,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (done) return true;
     if (i == 0) t0 = global_ns();
     else if ((i & 15) == 0 && global_ns() - t0 > kWaitNs) return false;
-    __nanosleep(32);
   }
 }
 
@@ -237,8 +240,12 @@ __device__ __forceinline__ float max64(const float (&v)[kTcTok]) {
                fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 template <int HD>
-__global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
+__global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 168 regs per SM partition
     prefix_kernel(const DecodeParams p, const PrefixParams pp,
                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
@@ -252,14 +259,18 @@ __global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
   const uint32_t v_ring = k_ring + kTcStages * Cfg::KV_BYTES;
   int* const s_phys = reinterpret_cast<int*>(gbase + Cfg::BODY);
   uint8_t* const tail = gbase + Cfg::BODY + pp.phys_bytes;
-  const uint32_t bar_s = smem_u32(tail);       // S of a tile is in tensor memory
-  const uint32_t bar_o = smem_u32(tail + 8);   // a tile's P V has been accumulated
-  const uint32_t bar_k = smem_u32(tail + 16);  // [2]: K tile (and, first, Q) landed
-  const uint32_t bar_v = smem_u32(tail + 32);  // [2]: V tile landed
-  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 48);
+  const uint32_t bar_sfull = smem_u32(tail);        // S of a tile is in tensor memory (MMA)
+  const uint32_t bar_sfree = smem_u32(tail + 8);    // every row has read S (4 warps)
+  const uint32_t bar_pfull = smem_u32(tail + 16);   // every row has written P (4 warps)
+  const uint32_t bar_odone = smem_u32(tail + 24);   // a tile's P V has been accumulated (MMA)
+  const uint32_t bar_k = smem_u32(tail + 32);       // [2]: K tile (and, first, Q) landed
+  const uint32_t bar_v = smem_u32(tail + 48);       // [2]: V tile landed
+  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 64);
+  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 68);
 
   const int kvh = blockIdx.x, split = blockIdx.y, rg = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid / kWarp;
+  const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
+  const bool producer = warp == kTcSoftmaxWarps;
   const int G = p.group;
   const int spc = kTcRows / G;  // sequences per CTA; rows (seq, head) = spc * G <= 128
   const int t0 = split * pp.pchunk;
@@ -268,7 +279,7 @@ __global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
   const int blk0 = t0 >> p.log2_bs;
   const int ntiles = (t1 - t0 + kTcTok - 1) / kTcTok;
 
-  // ---- set-up: block-table slice, barriers, tensor memory
+  // ---- set-up: block-table slice, barriers, tensor memory, zeroed Q padding
   {
     const int nphys = ((t1 - 1) >> p.log2_bs) - blk0 + 1;
     for (int i = tid; i < nphys; i += kTcThreads) {
@@ -281,12 +292,15 @@ __global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
     }
   }
   if (tid == 0) {
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sfree, kTcSoftmaxWarps);
+    mbar_init(bar_pfull, kTcSoftmaxWarps);
+    mbar_init(bar_odone, 1);
     mbar_init(bar_k, 1);
     mbar_init(bar_k + 8, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_v + 8, 1);
+    *s_fail = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -303,221 +317,248 @@ __global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
       *reinterpret_cast<uint4*>(gbase + db * Cfg::Q_DB + rr * 128 + (tid % 8) * 16) =
           make_uint4(0, 0, 0, 0);
   fence_async_smem();
-
-  // ---- this thread's row
-  const int row = tid;
-  const int seq = rg * spc + row / G;
-  const bool rvalid = row < spc * G && seq < p.num_seqs;
-  const size_t qrow = (size_t)(rvalid ? seq : 0) * p.num_q_heads + kvh * G + row % G;
-  int lim = 0;  // tokens of the prefix this row attends to
-  if (rvalid) {
-    int ctx = p.context_lens[seq];
-    ctx = ctx < 0 ? 0 : ctx;
-    lim = min(ctx, pp.prefix_len);
-  }
-
-  // ---- tile copies (thread 0): K or V tile j as boxes of R token rows x 64
-  // head_dim columns, one per (block piece, column block); a bad block, or
-  // rows past the slice, load from past the end of the cache: zeros
-  const int R = bs < kTcTok ? bs : kTcTok;
-  const int oob = p.num_blocks * bs;
-  auto load_tile = [&](const CUtensorMap* map, uint32_t stage, int j, uint32_t bar) {
-    mbar_expect_tx(bar, Cfg::KV_BYTES);
-    const int tt = t0 + j * kTcTok;
-    for (int b = 0; b < kTcTok / R; ++b) {
-      const int t = tt + b * R;
-      const int phys = t < t1 ? s_phys[(t >> p.log2_bs) - blk0] : -1;
-      const int z = phys >= 0 ? phys * bs + (t & (bs - 1)) : oob;
-#pragma unroll
-      for (int db = 0; db < Cfg::DB; ++db)
-        tma_load_3d(stage + (uint32_t)(db * Cfg::KV_DB + b * R * 128), map, db * 64, kvh, z, bar);
-    }
-  };
-  auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
-  auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
-
   tc_fence_before();
   __syncthreads();  // s_phys, barriers, tensor-memory address, zeroed Q rows
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-
-  constexpr uint32_t kIdQK = idesc_bf16(kTcRows, kTcTok, 0);
-  constexpr uint32_t kIdPV = idesc_bf16(kTcRows, HD, 1);
-  auto issue_qk = [&](int j) {  // S = Q K^T of tile j (thread 0)
-    const uint32_t kS = kstage(j);
-#pragma unroll
-    for (int ks = 0; ks < HD / 16; ++ks) {
-      const uint32_t koff = (uint32_t)((ks >> 2) * Cfg::KV_DB + (ks & 3) * 32);
-      const uint32_t qoff = (uint32_t)((ks >> 2) * Cfg::Q_DB + (ks & 3) * 32);
-      mma_ss(tmem + Cfg::S_COL, smem_desc(q_sm + qoff, 16, 1024), smem_desc(kS + koff, 16, 1024),
-             kIdQK, ks > 0);
-    }
-    mma_commit(bar_s);
-  };
-  auto issue_pv = [&](int j) {  // O += P V of tile j (thread 0)
-    const uint32_t vS = vstage(j);
-#pragma unroll
-    for (int kk = 0; kk < kTcTok / 16; ++kk) {
-      const uint64_t bd = smem_desc(vS + (uint32_t)(kk * 16 * 128), Cfg::KV_DB, 1024);
-      mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PH_COL + kk * 8, bd, kIdPV, (j > 0 || kk > 0));
-      mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PL_COL + kk * 8, bd, kIdPV, 1u);
-    }
-    mma_commit(bar_o);
-  };
-
-  // ---- prologue (thread 0): Q with K0, V0, K1, V1; then S of tile 0
   bool ok = true;
-  if (tid == 0) {
-    mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
-#pragma unroll
-    for (int db = 0; db < Cfg::DB; ++db)
-      tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
-    load_tile(&tm_k, kstage(0), 0, bar_k);
-    load_tile(&tm_v, vstage(0), 0, bar_v);
-    if (ntiles > 1) {
-      load_tile(&tm_k, kstage(1), 1, bar_k + 8);
-      load_tile(&tm_v, vstage(1), 1, bar_v + 8);
-    }
-    ok = mbar_wait(bar_k, 0);
-    tc_fence_after();
-    if (ok) issue_qk(0);
-  }
 
-  float m_ref = -CUDART_INF_F;  // reference maximum of this row (scaled, log2 units)
-  float l_run = 0.f;
-  bool failed = false;
-  const float sc = p.scale_log2;
-  for (int j = 0; j < ntiles; ++j) {
-    const int tt = t0 + j * kTcTok;
-    // ---- scores of tile j; its K stage takes tile j + 2
-    ok &= warp_wait(bar_s, (uint32_t)(j & 1));
-    tc_fence_after();
-    if (tid == 0 && j + 2 < ntiles) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
-    float s[kTcTok];
-    {
-      float a[32], b[32];
-      tmem_ld32(tmem + lane_base + Cfg::S_COL, a);
-      tmem_ld32(tmem + lane_base + Cfg::S_COL + 32, b);
-      tmem_wait_ld();
+  if (producer) {
+    // ================= producer: one lane issues every copy and MMA ==========
+    if (lane == 0) {
+      const int R = bs < kTcTok ? bs : kTcTok;  // token rows per box
+      const int nbox = kTcTok / R;
+      const int oob = p.num_blocks * bs;
+      // K or V tile j as boxes of R token rows x 64 head_dim columns, one per
+      // (block piece, column block); a bad block, or rows past the slice, load
+      // from past the end of the cache: zeros
+      auto load_tile = [&](const CUtensorMap* map, uint32_t stage, int j, uint32_t bar) {
+        const int tt = t0 + j * kTcTok;
+        constexpr int kMaxBox = kTcTok / 8;  // block_size >= 8
+        int z[kMaxBox];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        s[i] = a[i];
-        s[32 + i] = b[i];
-      }
-    }
-    // valid tokens of this row: inside the slice, below the row's limit, in a good block
-    const int nval = max(0, min(t1, lim) - tt);
-    bool bad = false;
-    for (int b = (tt >> p.log2_bs) - blk0; b <= ((min(tt + kTcTok, t1) - 1) >> p.log2_bs) - blk0;
-         ++b)
-      bad |= s_phys[b] < 0;
-    if (nval < kTcTok || bad || sc <= 0.f) {  // masked tile (or an unusual scale): the slow path
+        for (int b = 0; b < kMaxBox; ++b) {
+          const int t = tt + b * R;
+          const int phys = (b < nbox && t < t1) ? s_phys[(t >> p.log2_bs) - blk0] : -1;
+          z[b] = phys >= 0 ? phys * bs + (t & (bs - 1)) : oob;
+        }
+        mbar_expect_tx(bar, Cfg::KV_BYTES);
 #pragma unroll
-      for (int i = 0; i < kTcTok; ++i) {
-        bool v = i < nval;
-        if (bad) v = v && s_phys[((tt + i) >> p.log2_bs) - blk0] >= 0;
-        s[i] = v ? s[i] * sc : -CUDART_INF_F;
-      }
-    } else {
+        for (int b = 0; b < kMaxBox; ++b)
+          if (b < nbox)
 #pragma unroll
-      for (int i = 0; i < kTcTok; ++i) s[i] *= sc;
-    }
-    const float mt = max64(s);
-    const bool move = mt > m_ref + kRescaleLog2;  // also true for the first valid tile
-    const float m_new = move ? mt : m_ref;
-    const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
+            for (int db = 0; db < Cfg::DB; ++db)
+              tma_load_3d(stage + (uint32_t)(db * Cfg::KV_DB + b * R * 128), map, db * 64, kvh,
+                          z[b], bar);
+      };
+      auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
+      auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
+      // descriptors of the operand bases; an MMA adds its offset (>> 4) to the
+      // start-address field, which never carries out (shared addresses < 256 KB)
+      const uint64_t dq = smem_desc(q_sm, 16, 1024);
+      const uint64_t dk = smem_desc(k_ring, 16, 1024);
+      const uint64_t dv = smem_desc(v_ring, Cfg::KV_DB, 1024);
+      constexpr uint32_t kIdQK = idesc_bf16(kTcRows, kTcTok, 0);
+      constexpr uint32_t kIdPV = idesc_bf16(kTcRows, HD, 1);
+      auto issue_qk = [&](int j) {  // S = Q K^T of tile j
+        const uint64_t kb0 = dk + (uint64_t)(((j % kTcStages) * Cfg::KV_BYTES) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < HD / 16; ++ks) {
+          const uint32_t koff = (uint32_t)((ks >> 2) * Cfg::KV_DB + (ks & 3) * 32) >> 4;
+          const uint32_t qoff = (uint32_t)((ks >> 2) * Cfg::Q_DB + (ks & 3) * 32) >> 4;
+          mma_ss(tmem + Cfg::S_COL, dq + qoff, kb0 + koff, kIdQK, ks > 0);
+        }
+        mma_commit(bar_sfull);
+      };
+      auto issue_pv = [&](int j) {  // O += P V of tile j
+        const uint64_t vb0 = dv + (uint64_t)(((j % kTcStages) * Cfg::KV_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kTcTok / 16; ++kk) {
+          const uint64_t bd = vb0 + (uint64_t)((kk * 16 * 128) >> 4);
+          mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PH_COL + kk * 8, bd, kIdPV, (j > 0 || kk > 0));
+          mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PL_COL + kk * 8, bd, kIdPV, 1u);
+        }
+        mma_commit(bar_odone);
+      };
 
-    // ---- the previous tile's P V must be done: P is overwritten, O may be
-    // rescaled, and its V stage takes tile j + 1
-    if (j > 0) {
-      ok &= warp_wait(bar_o, (uint32_t)((j - 1) & 1));
+      // Q with K0, V0, K1, V1; then S of tile 0
+      mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
+#pragma unroll
+      for (int db = 0; db < Cfg::DB; ++db)
+        tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
+      load_tile(&tm_k, kstage(0), 0, bar_k);
+      load_tile(&tm_v, vstage(0), 0, bar_v);
+      if (ntiles > 1) {
+        load_tile(&tm_k, kstage(1), 1, bar_k + 8);
+        load_tile(&tm_v, vstage(1), 1, bar_v + 8);
+      }
+      ok = mbar_wait(bar_k, 0);
       tc_fence_after();
-      if (tid == 0 && j + 1 < ntiles) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
+      if (ok) issue_qk(0);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        // every row has read S_j: S of tile j + 1 may overwrite it, and K tile
+        // j's stage (its S is done) takes tile j + 2
+        ok = mbar_wait(bar_sfree, (uint32_t)(j & 1));
+        tc_fence_after();
+        if (ok && j + 1 < ntiles) {
+          ok = mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
+          if (ok) issue_qk(j + 1);
+        }
+        if (ok && j + 2 < ntiles) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
+        // P V of tile j - 1 is done: its V stage takes tile j + 1
+        if (ok && j > 0) {
+          ok = mbar_wait(bar_odone, (uint32_t)((j - 1) & 1));
+          if (ok && j + 1 < ntiles) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
+        }
+        // every row has written P_j, V_j has landed: O += P_j V_j
+        if (ok) ok = mbar_wait(bar_pfull, (uint32_t)(j & 1));
+        if (ok) ok = mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
+        tc_fence_after();
+        if (ok) issue_pv(j);
+      }
+      if (!ok) *s_fail = 1;
     }
-    // rare: rescale O in place.  tcgen05.ld/st are warp-collective, so the whole
-    // warp takes this path when any of its rows needs it (alpha = 1 for the rest).
-    const bool need = move && j > 0 && m_ref != -CUDART_INF_F;
-    if (__any_sync(0xffffffffu, need)) {
-      const float a_row = need ? alpha : 1.f;
+  } else {
+    // ================= softmax: thread r owns row r ==========================
+    const int row = tid;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int seq = rg * spc + row / G;
+    const bool rvalid = row < spc * G && seq < p.num_seqs;
+    const size_t qrow = (size_t)(rvalid ? seq : 0) * p.num_q_heads + kvh * G + row % G;
+    int lim = 0;  // tokens of the prefix this row attends to
+    if (rvalid) {
+      int ctx = p.context_lens[seq];
+      ctx = ctx < 0 ? 0 : ctx;
+      lim = min(ctx, pp.prefix_len);
+    }
+    float m_ref = -CUDART_INF_F;  // reference maximum of this row (scaled, log2 units)
+    float l_run = 0.f;
+    const float sc = p.scale_log2;
+    for (int j = 0; j < ntiles; ++j) {
+      const int tt = t0 + j * kTcTok;
+      // ---- scores of tile j, then release S to the next tile's MMA
+      ok = ok && warp_wait(bar_sfull, (uint32_t)(j & 1));
+      tc_fence_after();
+      float s[kTcTok];
+      {
+        float a[32], b[32];
+        tmem_ld32(tmem + lane_base + Cfg::S_COL, a);
+        tmem_ld32(tmem + lane_base + Cfg::S_COL + 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          s[i] = a[i];
+          s[32 + i] = b[i];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sfree);
+      // valid tokens of this row: inside the slice, below the row's limit, in a good block
+      const int nval = max(0, min(t1, lim) - tt);
+      bool bad = false;
+      for (int b = (tt >> p.log2_bs) - blk0; b <= ((min(tt + kTcTok, t1) - 1) >> p.log2_bs) - blk0;
+           ++b)
+        bad |= s_phys[b] < 0;
+      if (nval < kTcTok || bad || sc <= 0.f) {  // masked tile (or an unusual scale)
+#pragma unroll
+        for (int i = 0; i < kTcTok; ++i) {
+          bool v = i < nval;
+          if (bad) v = v && s_phys[((tt + i) >> p.log2_bs) - blk0] >= 0;
+          s[i] = v ? s[i] * sc : -CUDART_INF_F;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTcTok; ++i) s[i] *= sc;
+      }
+      const float mt = max64(s);
+      const bool move = mt > m_ref + kRescaleLog2;  // also true for the first valid tile
+      const float m_new = move ? mt : m_ref;
+      const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
+
+      // ---- the previous tile's P V must be done: P is overwritten, O may be rescaled
+      if (j > 0) {
+        ok = ok && warp_wait(bar_odone, (uint32_t)((j - 1) & 1));
+        tc_fence_after();
+      }
+      // rare: rescale O in place.  tcgen05.ld/st are warp-collective, so the whole
+      // warp takes this path when any of its rows needs it (alpha = 1 for the rest).
+      const bool need = move && j > 0 && m_ref != -CUDART_INF_F;
+      if (__any_sync(0xffffffffu, need)) {
+        const float a_row = need ? alpha : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < HD; c += 32) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o);
+          tmem_wait_ld();
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * a_row);
+          tmem_st32(tmem + lane_base + Cfg::O_COL + c, w);
+          tmem_wait_st();
+        }
+      }
+      l_run *= alpha;
+      m_ref = m_new;
+      const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
+
+      // ---- P = 2^(s - m) as bf16 hi + lo, into tensor memory (8 partial sums)
+      {
+        uint32_t hi[32], lo[32];
+        float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = fast_exp2(s[2 * i] - m_use), x1 = fast_exp2(s[2 * i + 1] - m_use);
+          rs[i & 7] += x0 + x1;
+          const uint32_t h = pack_bf16(x0, x1);
+          const float2 f = unpack_bf16(h);
+          hi[i] = h;
+          lo[i] = pack_bf16(x0 - f.x, x1 - f.y);
+        }
+        l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        tmem_st32(tmem + lane_base + Cfg::PH_COL, hi);
+        tmem_st32(tmem + lane_base + Cfg::PL_COL, lo);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull);
+      if (!ok) break;
+    }
+    // ---- the last P V
+    ok = ok && warp_wait(bar_odone, (uint32_t)((ntiles - 1) & 1));
+    tc_fence_after();
+    if (!ok) *s_fail = 1;
+    // ---- normalise this slice's partial into shared memory (the K/V rings,
+    // idle once the last P V is done), so that whole rows go out coalesced
+    if (ok) {
+      constexpr int CHK = HD / 4;  // 16-byte chunks per row
+      float4* stage = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES);
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < HD; c += 32) {
         float o[32];
         tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o);
         tmem_wait_ld();
-        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * a_row);
-        tmem_st32(tmem + lane_base + Cfg::O_COL + c, w);
-        tmem_wait_st();
+        for (int i = 0; i < 8; ++i) {
+          const int ch = c / 4 + i;
+          stage[row * CHK + (ch ^ (row & (CHK - 1)))] = make_float4(
+              o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+        }
       }
-    }
-    l_run *= alpha;
-    m_ref = m_new;
-    const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
-
-    // ---- P = 2^(s - m) as bf16 hi + lo, into tensor memory (8 partial sums)
-    {
-      uint32_t hi[32], lo[32];
-      float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float x0 = fast_exp2(s[2 * i] - m_use), x1 = fast_exp2(s[2 * i + 1] - m_use);
-        rs[i & 7] += x0 + x1;
-        const uint32_t h = pack_bf16(x0, x1);
-        const float2 f = unpack_bf16(h);
-        hi[i] = h;
-        lo[i] = pack_bf16(x0 - f.x, x1 - f.y);
-      }
-      l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-      tmem_st32(tmem + lane_base + Cfg::PH_COL, hi);
-      tmem_st32(tmem + lane_base + Cfg::PL_COL, lo);
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    failed = __syncthreads_or(!ok);
-    if (failed) break;
-    if (tid == 0) {  // V tile j and K tile j + 1 landed -> P V of tile j, S of tile j + 1
-      ok &= mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
-      tc_fence_after();
-      if (ok) issue_pv(j);
-      if (ok && j + 1 < ntiles) {
-        ok &= mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
-        if (ok) issue_qk(j + 1);
-      }
+      if (rvalid)
+        p.ws_lse[qrow * p.ws_slots + split] = l_run > 0.f ? m_ref + log2f(l_run) : -CUDART_INF_F;
     }
   }
 
-  // ---- the last P V, then normalise this slice's partial.  Thread r holds
-  // row r; the rows go through shared memory (the K/V rings, now idle) so that
-  // each warp writes whole rows of the workspace.
-  if (!failed) {
-    ok &= warp_wait(bar_o, (uint32_t)((ntiles - 1) & 1));
-    tc_fence_after();
-    failed = __syncthreads_or(!ok);
-  }
-  if (!failed) {
-    constexpr int CHK = HD / 4;  // 16-byte chunks per row
-    float4* stage = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES);
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll 1
-    for (int c = 0; c < HD; c += 32) {
-      float o[32];
-      tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int ch = c / 4 + i;
-        stage[row * CHK + (ch ^ (row & (CHK - 1)))] =
-            make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
-      }
-    }
-    if (rvalid)
-      p.ws_lse[qrow * p.ws_slots + split] = l_run > 0.f ? m_ref + log2f(l_run) : -CUDART_INF_F;
-    __syncthreads();
+  tc_fence_before();
+  const bool failed = __syncthreads_or(!ok || *s_fail);
+  if (!failed && !producer) {  // coalesced rows of the workspace
+    constexpr int CHK = HD / 4;
     constexpr int RPI = 32 / CHK;  // rows per warp store
-    const int lane = tid & 31;
-    for (int rr = warp * RPI + lane / CHK; rr < kTcRows; rr += 4 * RPI) {
+    const float4* stage = reinterpret_cast<const float4*>(gbase + Cfg::Q_BYTES);
+    for (int rr = warp * RPI + lane / CHK; rr < kTcRows; rr += kTcSoftmaxWarps * RPI) {
       const int sq = rg * spc + rr / G;
       if (rr >= spc * G || sq >= p.num_seqs) continue;
       const size_t slot = ((size_t)sq * p.num_q_heads + kvh * G + rr % G) * p.ws_slots + split;
@@ -525,8 +566,6 @@ __global__ void __maxnreg__(192)  // 2 CTAs x 128 threads per SM
       reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] = stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
     }
   }
-  tc_fence_before();
-  failed = __syncthreads_or(failed);
   if (failed && tid == 0) set_flag(p.err_flag, PKV_FLAG_TIMEOUT);
   if (warp == 0) {
     tc_fence_after();
@@ -571,7 +610,7 @@ cudaError_t bf16_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
 
 template <int HD>
 int smem_bytes(const PrefixParams& pp) {
-  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 64;
+  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 128;
 }
 
 template <int HD>
