@@ -27,9 +27,10 @@
 // The running maximum is only moved when a tile's maximum exceeds it by more
 // than 2^8 (then O is rescaled in tensor memory): exponentials stay below 256,
 // and the final normalisation uses the same maximum as every P, so the result
-// is the same softmax.  A fifth warp is the producer: one of its lanes issues
-// every copy and MMA; copies, tcgen05.commit and the softmax warps' hand-offs
-// (S read, P written) arrive on mbarriers, each wait bounded.  Q, K and V move by
+// is the same softmax.  Two more warps feed the tensor cores: one lane of a
+// copy warp issues every TMA copy, one lane of an MMA warp every tcgen05.mma;
+// copies, tcgen05.commit and the softmax warps' hand-offs (S read, P written)
+// arrive on mbarriers, each wait bounded.  Q, K and V move by
 // TMA (cp.async.bulk.tensor) straight into the 128-byte-swizzled layout the
 // MMAs read: Q as a (sequences x heads x 64 columns) box, the K and V tiles
 // as one box per paged block (or 64-token piece of one) and column block, a
@@ -57,7 +58,7 @@ namespace pkv {
 namespace {
 
 constexpr int kTcSoftmaxWarps = 4;  // thread r owns row r; warp w reads TMEM lanes 32w..32w+31
-constexpr int kTcThreads = (kTcSoftmaxWarps + 1) * 32;  // plus one producer warp
+constexpr int kTcThreads = (kTcSoftmaxWarps + 2) * 32;  // plus a copy warp and an MMA warp
 constexpr int kTcRows = 128;     // rows per CTA (MMA M)
 constexpr int kTcTok = kPrefixTokens;  // tokens per tile (MMA N of Q K^T)
 constexpr int kTcStages = 2;
@@ -245,7 +246,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 }
 
 template <int HD>
-__global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 168 regs per SM partition
+__global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs per SM partition
     prefix_kernel(const DecodeParams p, const PrefixParams pp,
                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
@@ -260,17 +261,18 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
   int* const s_phys = reinterpret_cast<int*>(gbase + Cfg::BODY);
   uint8_t* const tail = gbase + Cfg::BODY + pp.phys_bytes;
   const uint32_t bar_sfull = smem_u32(tail);        // S of a tile is in tensor memory (MMA)
-  const uint32_t bar_sfree = smem_u32(tail + 8);    // every row has read S (4 warps)
+  const uint32_t bar_sfree = smem_u32(tail + 8);    // every row has read S (4 warps; MMA warp)
   const uint32_t bar_pfull = smem_u32(tail + 16);   // every row has written P (4 warps)
   const uint32_t bar_odone = smem_u32(tail + 24);   // a tile's P V has been accumulated (MMA)
   const uint32_t bar_k = smem_u32(tail + 32);       // [2]: K tile (and, first, Q) landed
   const uint32_t bar_v = smem_u32(tail + 48);       // [2]: V tile landed
-  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 64);
-  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 68);
+  const uint32_t bar_sfree_c = smem_u32(tail + 64);  // the same, waited by the copy warp
+  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 72);
+  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 76);
 
   const int kvh = blockIdx.x, split = blockIdx.y, rg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
-  const bool producer = warp == kTcSoftmaxWarps;
+  const bool copier = warp == kTcSoftmaxWarps, mma_warp = warp == kTcSoftmaxWarps + 1;
   const int G = p.group;
   const int spc = kTcRows / G;  // sequences per CTA; rows (seq, head) = spc * G <= 128
   const int t0 = split * pp.pchunk;
@@ -294,6 +296,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
   if (tid == 0) {
     mbar_init(bar_sfull, 1);
     mbar_init(bar_sfree, kTcSoftmaxWarps);
+    mbar_init(bar_sfree_c, kTcSoftmaxWarps);
     mbar_init(bar_pfull, kTcSoftmaxWarps);
     mbar_init(bar_odone, 1);
     mbar_init(bar_k, 1);
@@ -323,8 +326,10 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
   const uint32_t tmem = *s_tmem;
   bool ok = true;
 
-  if (producer) {
-    // ================= producer: one lane issues every copy and MMA ==========
+  if (copier) {
+    // ================= copy warp: one lane issues every TMA copy =============
+    // (each waiter has barriers of its own, so that no waiter can fall two
+    // phases behind the barrier it polls)
     if (lane == 0) {
       const int R = bs < kTcTok ? bs : kTcTok;  // token rows per box
       const int nbox = kTcTok / R;
@@ -353,6 +358,34 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
       };
       auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
       auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
+      // Q with K0 first (S of tile 0 waits for them), then V0, K1, V1
+      mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
+#pragma unroll
+      for (int db = 0; db < Cfg::DB; ++db)
+        tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
+      load_tile(&tm_k, kstage(0), 0, bar_k);
+      load_tile(&tm_v, vstage(0), 0, bar_v);
+      if (ntiles > 1) {
+        load_tile(&tm_k, kstage(1), 1, bar_k + 8);
+        load_tile(&tm_v, vstage(1), 1, bar_v + 8);
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        // every row has read S_j, so its MMA is done: K tile j's stage takes tile j + 2
+        if (j + 2 < ntiles) {
+          ok = mbar_wait(bar_sfree_c, (uint32_t)(j & 1));
+          if (ok) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
+        }
+        // P V of tile j - 1 is done: its V stage takes tile j + 1
+        if (ok && j > 0 && j + 1 < ntiles) {
+          ok = mbar_wait(bar_odone, (uint32_t)((j - 1) & 1));
+          if (ok) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
+        }
+      }
+      if (!ok) *s_fail = 1;
+    }
+  } else if (mma_warp) {
+    // ================= MMA warp: one lane issues every tcgen05.mma ============
+    if (lane == 0) {
       // descriptors of the operand bases; an MMA adds its offset (>> 4) to the
       // start-address field, which never carries out (shared addresses < 256 KB)
       const uint64_t dq = smem_desc(q_sm, 16, 1024);
@@ -380,35 +413,16 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
         }
         mma_commit(bar_odone);
       };
-
-      // Q with K0, V0, K1, V1; then S of tile 0
-      mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
-#pragma unroll
-      for (int db = 0; db < Cfg::DB; ++db)
-        tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
-      load_tile(&tm_k, kstage(0), 0, bar_k);
-      load_tile(&tm_v, vstage(0), 0, bar_v);
-      if (ntiles > 1) {
-        load_tile(&tm_k, kstage(1), 1, bar_k + 8);
-        load_tile(&tm_v, vstage(1), 1, bar_v + 8);
-      }
       ok = mbar_wait(bar_k, 0);
       tc_fence_after();
       if (ok) issue_qk(0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        // every row has read S_j: S of tile j + 1 may overwrite it, and K tile
-        // j's stage (its S is done) takes tile j + 2
+        // every row has read S_j: S of tile j + 1 may overwrite it
         ok = mbar_wait(bar_sfree, (uint32_t)(j & 1));
         tc_fence_after();
         if (ok && j + 1 < ntiles) {
           ok = mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
           if (ok) issue_qk(j + 1);
-        }
-        if (ok && j + 2 < ntiles) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
-        // P V of tile j - 1 is done: its V stage takes tile j + 1
-        if (ok && j > 0) {
-          ok = mbar_wait(bar_odone, (uint32_t)((j - 1) & 1));
-          if (ok && j + 1 < ntiles) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
         }
         // every row has written P_j, V_j has landed: O += P_j V_j
         if (ok) ok = mbar_wait(bar_pfull, (uint32_t)(j & 1));
@@ -453,7 +467,10 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree);
+      if (lane == 0) {
+        mbar_arrive(bar_sfree);
+        mbar_arrive(bar_sfree_c);
+      }
       // valid tokens of this row: inside the slice, below the row's limit, in a good block
       const int nval = max(0, min(t1, lim) - tt);
       bool bad = false;
@@ -554,7 +571,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 5 warps per SM: at most 3 warps x 
 
   tc_fence_before();
   const bool failed = __syncthreads_or(!ok || *s_fail);
-  if (!failed && !producer) {  // coalesced rows of the workspace
+  if (!failed && warp < kTcSoftmaxWarps) {  // coalesced rows of the workspace
     constexpr int CHK = HD / 4;
     constexpr int RPI = 32 / CHK;  // rows per warp store
     const float4* stage = reinterpret_cast<const float4*>(gbase + Cfg::Q_BYTES);
