@@ -107,7 +107,9 @@ PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head
   const long long target = 2LL * sm_count();
   long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
   const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;
+  const int min_ps = (prefix_len + pkv::kMaxPrefixChunk - 1) / pkv::kMaxPrefixChunk;
   if (ps > max_ps) ps = max_ps;
+  if (ps < min_ps) ps = min_ps;  // bounds the block-table slice in shared memory
   if (ps < 1) ps = 1;
   pl.pchunk = round_up((int)((prefix_len + ps - 1) / ps), pkv::kPrefixTokens);
   pl.ps = (prefix_len + pl.pchunk - 1) / pl.pchunk;

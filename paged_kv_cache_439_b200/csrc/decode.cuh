@@ -44,8 +44,8 @@ struct PrefixParams {
   int rows;           // q rows per KV head: num_seqs * group
   int phys_bytes;     // shared-memory bytes for one slice's block-table entries
 };
-constexpr int kPrefixWarps = 4;    // 16 q rows per warp
 constexpr int kPrefixTokens = 64;  // tokens per shared-memory stage
+constexpr int kMaxPrefixChunk = 8192;  // prefix tokens per slice at most
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
                           cudaStream_t st);

@@ -29,19 +29,20 @@
 // and the final normalisation uses the same maximum as every P, so the result
 // is the same softmax.  Two more warps feed the tensor cores: one lane of a
 // copy warp issues every TMA copy, one lane of an MMA warp every tcgen05.mma;
-// copies, tcgen05.commit and the softmax warps' hand-offs (S read, P written)
-// arrive on mbarriers, each wait bounded.  Q, K and V move by
+// copies, tcgen05.commit (S ready, P V done, and per ring stage "K/V stage
+// free") and the softmax warps' hand-offs (S read, P written) arrive on
+// mbarriers, each wait bounded.  Q, K and V move by
 // TMA (cp.async.bulk.tensor) straight into the 128-byte-swizzled layout the
 // MMAs read: Q as a (sequences x heads x 64 columns) box, the K and V tiles
 // as one box per paged block (or 64-token piece of one) and column block, a
 // bad block being read from past the end of the cache (zero fill).  K and V
 // have two-stage rings of their own.  Once every row has read S of tile j
-// into registers, S of tile j + 1 is issued (it runs during tile j's softmax)
-// and K tile j + 2 is fetched; V tile j + 1 is fetched once P V of tile j - 1
-// is done.  Two CTAs share an SM (half of its tensor memory each, at most 168
-// registers a thread so that both fit), so one CTA's softmax overlaps the
-// other's MMAs.  The softmax keeps eight independent max and
-// sum chains per row.
+// into registers, S of tile j + 1 is issued (it runs during tile j's
+// softmax); K tile j + 2 is fetched once S of tile j is done, V tile j + 1
+// once P V of tile j - 1 is done.  Two CTAs share an SM (half of its tensor
+// memory each, at most 168 registers a thread so that both fit), so one CTA's
+// softmax overlaps the other's MMAs.  The softmax keeps eight independent max
+// and sum chains per row.
 #include <math_constants.h>
 
 #include <cuda.h>
@@ -260,15 +261,19 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
   const uint32_t v_ring = k_ring + kTcStages * Cfg::KV_BYTES;
   int* const s_phys = reinterpret_cast<int*>(gbase + Cfg::BODY);
   uint8_t* const tail = gbase + Cfg::BODY + pp.phys_bytes;
+  // Each barrier's waiters must never fall two phases behind it (try_wait.parity
+  // would then match the incomplete phase two ahead): every waiter polls a
+  // barrier whose next phase cannot complete before that waiter's own next step.
   const uint32_t bar_sfull = smem_u32(tail);        // S of a tile is in tensor memory (MMA)
   const uint32_t bar_sfree = smem_u32(tail + 8);    // every row has read S (4 warps; MMA warp)
   const uint32_t bar_pfull = smem_u32(tail + 16);   // every row has written P (4 warps)
   const uint32_t bar_odone = smem_u32(tail + 24);   // a tile's P V has been accumulated (MMA)
   const uint32_t bar_k = smem_u32(tail + 32);       // [2]: K tile (and, first, Q) landed
   const uint32_t bar_v = smem_u32(tail + 48);       // [2]: V tile landed
-  const uint32_t bar_sfree_c = smem_u32(tail + 64);  // the same, waited by the copy warp
-  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 72);
-  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 76);
+  const uint32_t bar_kfree = smem_u32(tail + 64);   // [2]: S of the stage's K tile is done
+  const uint32_t bar_vfree = smem_u32(tail + 80);   // [2]: P V of the stage's V tile is done
+  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 96);
+  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 100);
 
   const int kvh = blockIdx.x, split = blockIdx.y, rg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
@@ -296,7 +301,10 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
   if (tid == 0) {
     mbar_init(bar_sfull, 1);
     mbar_init(bar_sfree, kTcSoftmaxWarps);
-    mbar_init(bar_sfree_c, kTcSoftmaxWarps);
+    mbar_init(bar_kfree, 1);
+    mbar_init(bar_kfree + 8, 1);
+    mbar_init(bar_vfree, 1);
+    mbar_init(bar_vfree + 8, 1);
     mbar_init(bar_pfull, kTcSoftmaxWarps);
     mbar_init(bar_odone, 1);
     mbar_init(bar_k, 1);
@@ -328,8 +336,9 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
 
   if (copier) {
     // ================= copy warp: one lane issues every TMA copy =============
-    // (each waiter has barriers of its own, so that no waiter can fall two
-    // phases behind the barrier it polls)
+    // It waits only on per-stage "free" barriers: the next phase of each needs
+    // the tile this warp loads after the wait, so the warp can never be two
+    // phases behind one (which would alias the parity it polls).
     if (lane == 0) {
       const int R = bs < kTcTok ? bs : kTcTok;  // token rows per box
       const int nbox = kTcTok / R;
@@ -370,14 +379,14 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
         load_tile(&tm_v, vstage(1), 1, bar_v + 8);
       }
       for (int j = 0; ok && j < ntiles; ++j) {
-        // every row has read S_j, so its MMA is done: K tile j's stage takes tile j + 2
+        // S of tile j is done: K tile j's stage takes tile j + 2
         if (j + 2 < ntiles) {
-          ok = mbar_wait(bar_sfree_c, (uint32_t)(j & 1));
+          ok = mbar_wait(bar_kfree + 8 * (j % 2), (uint32_t)((j / 2) & 1));
           if (ok) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
         }
         // P V of tile j - 1 is done: its V stage takes tile j + 1
         if (ok && j > 0 && j + 1 < ntiles) {
-          ok = mbar_wait(bar_odone, (uint32_t)((j - 1) & 1));
+          ok = mbar_wait(bar_vfree + 8 * ((j - 1) % 2), (uint32_t)(((j - 1) / 2) & 1));
           if (ok) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
         }
       }
@@ -402,6 +411,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
           mma_ss(tmem + Cfg::S_COL, dq + qoff, kb0 + koff, kIdQK, ks > 0);
         }
         mma_commit(bar_sfull);
+        mma_commit(bar_kfree + 8 * (j % 2));
       };
       auto issue_pv = [&](int j) {  // O += P V of tile j
         const uint64_t vb0 = dv + (uint64_t)(((j % kTcStages) * Cfg::KV_BYTES) >> 4);
@@ -412,6 +422,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
           mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PL_COL + kk * 8, bd, kIdPV, 1u);
         }
         mma_commit(bar_odone);
+        mma_commit(bar_vfree + 8 * (j % 2));
       };
       ok = mbar_wait(bar_k, 0);
       tc_fence_after();
@@ -467,10 +478,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar_sfree);
-        mbar_arrive(bar_sfree_c);
-      }
+      if (lane == 0) mbar_arrive(bar_sfree);
       // valid tokens of this row: inside the slice, below the row's limit, in a good block
       const int nval = max(0, min(t1, lim) - tt);
       bool bad = false;
@@ -630,24 +638,30 @@ int smem_bytes(const PrefixParams& pp) {
   return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 128;
 }
 
+// Once per device: the kernel's dynamic shared-memory limit.
+template <int HD>
+cudaError_t prepare(int dev) {
+  static std::atomic<uint64_t> ready{0};
+  const uint64_t bit = 1ull << (dev & 63);
+  if (ready.load() & bit) return cudaSuccess;
+  int max_optin = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(prefix_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           max_optin);
+  if (e != cudaSuccess) return e;
+  ready.fetch_or(bit);
+  return cudaSuccess;
+}
+
 template <int HD>
 cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, cudaStream_t st) {
   const int smem = smem_bytes<HD>(pp);
-  auto k = prefix_kernel<HD>;
-  // opt in to the largest dynamic shared memory once per device
-  static std::atomic<uint64_t> ready{0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(ready.load() & bit)) {
-    int max_optin = 0;
-    e = cudaDeviceGetAttribute(&max_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin);
-    if (e != cudaSuccess) return e;
-    ready.fetch_or(bit);
-  }
+  e = prepare<HD>(dev);
+  if (e != cudaSuccess) return e;
   const int G = p.group;
   const int spc = kTcRows / G;
   const int rows_box = p.block_size < kTcTok ? p.block_size : kTcTok;
@@ -660,7 +674,7 @@ cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, cudaStream_t s
     e = bf16_map(&tv, p.v_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_kv_heads, pp.prefix_splits, (p.num_seqs + spc - 1) / spc);
-  k<<<grid, kTcThreads, smem, st>>>(p, pp, tq, tk, tv);
+  prefix_kernel<HD><<<grid, kTcThreads, smem, st>>>(p, pp, tq, tk, tv);
   return cudaGetLastError();
 }
 

@@ -119,3 +119,17 @@ def test_running_max_moves_inside_the_prefix():
     for splits in (0, 1):
         assert_close(_cascade(g, wl, prefix, num_splits=splits), ref, tol_for(wl), "moving max")
     assert g.flags() == 0
+
+
+def test_repeated_calls_never_stall():
+    """Many back-to-back calls, all split choices: the pipeline's hand-offs must
+    never deadlock (a stalled CTA gives up after 2 s and sets PKV_FLAG_TIMEOUT)."""
+    wl = make_workload("shared-prefix")
+    g = GpuCache(wl).fill()
+    q, bt, cl = wl.q.cuda(), wl.block_tables.cuda(), wl.context_lens.cuda()
+    for it in range(60):
+        pkv.paged_attention_decode_shared_prefix(
+            q, g.k, g.v, bt, cl, 4096, softmax_scale=wl.softmax_scale,
+            max_context_len=wl.max_context_len, num_splits=it % 3, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert g.flags() == 0
