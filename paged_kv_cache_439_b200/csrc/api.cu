@@ -43,9 +43,13 @@ int min_splits(int max_ctx) { return max_ctx <= 0 ? 1 : (max_ctx + kMaxChunk - 1
 //    only adds partial results to merge.  Keep S = 1 unless the last wave would
 //    run under half full with fewer than two waves in total, then take the
 //    smallest S that fixes that.
-//  * U < R / 2 (few, long sequences): cut the context so that about four CTAs
-//    per resident slot exist, which also evens out unequal context lengths;
-//    no split shorter than kMinChunk tokens.
+//  * U < R / 2 (few, long sequences): cut the context so that about
+//    kCtasPerSlot CTAs per resident slot exist, which also evens out unequal
+//    context lengths; no split shorter than kMinChunk tokens.  Among the
+//    counts from half to twice that target, take the smallest whose U * S
+//    CTAs fill their last wave at least 90% (equal-length contexts), else the
+//    best-filled one: 128 units on 444 slots take S = 10 (2.9 waves) rather
+//    than 14 (4.04 waves, the fifth nearly empty).
 int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_dtype cache_dt) {
   if (max_ctx <= 0 || num_seqs <= 0) return 1;
   const long long units = (long long)num_seqs * num_kv_heads;
@@ -62,7 +66,24 @@ int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_d
       if (full_waves >= 2 || rest == 0 || 2 * rest >= slots) break;
     }
   } else {
-    want = (kCtasPerSlot * slots + units - 1) / units;
+    const long long target = (kCtasPerSlot * slots + units - 1) / units;
+    long long best = target;
+    double best_fill = -1.0;
+    for (long long s = (target + 1) / 2; s <= 2 * target; ++s) {
+      if (s < lo || s > hi) continue;
+      const long long ctas = units * s;
+      const long long waves = (ctas + slots - 1) / slots;
+      const double fill = (double)ctas / (double)(waves * slots);
+      if (fill >= 0.9) {
+        best = s;
+        break;
+      }
+      if (fill > best_fill) {
+        best_fill = fill;
+        best = s;
+      }
+    }
+    want = best;
   }
   if (want > hi) want = hi;
   if (want < lo) want = lo;
