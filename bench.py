@@ -1,9 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of one paged-KV decode step on B200.
 
-A step is the whole hot path over one batch: ``kv_cache_append`` of each
-sequence's new token, then ``paged_attention_decode`` over every sequence's
-context (split-K plus merge when the planner splits).  Inputs are seeded
+A step is the whole hot path over one batch: each sequence's new token is
+appended to the cache, then every sequence attends over its context (split-K
+plus merge when the planner splits).  By default the step is one call,
+``paged_attention_decode_append`` (the append runs inside the decode kernel);
+``--unfused`` times ``kv_cache_append`` followed by ``paged_attention_decode``.  Inputs are seeded
 synthetic tensors shaped like the named workload and resident in HBM before
 the timed region.
 
@@ -57,6 +59,9 @@ def parse():
                     help="override the workload's KV-cache format")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix workload: read the shared blocks once per KV head")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the step as two calls (kv_cache_append, then decode) instead of "
+                         "the one-launch paged_attention_decode_append")
     ap.add_argument("--swap", action="store_true",
                     help="time swapping every sequence's blocks out to pinned host memory and "
                          "back (pkv_copy_blocks) against a plain pinned memcpy of the same bytes")
@@ -263,7 +268,11 @@ def config_dict(wl, args, splits):
         "head_dim": wl.head_dim, "block_size": wl.block_size, "cache_dtype": wl.cache_dtype,
         "num_blocks": wl.num_blocks, "num_splits": splits,
         "shared_prefix_pass": bool(getattr(args, "cascade", False)),
-        "step": "kv_cache_append (1 new token per sequence) + paged_attention_decode",
+        "step": ("kv_cache_append (1 new token per sequence) + paged_attention_decode"
+                 if (getattr(args, "cascade", False) or getattr(args, "unfused", False)
+                     or wl.cache_dtype == "f32") else
+                 "paged_attention_decode_append (1 new token per sequence appended inside "
+                 "the decode kernel)"),
         "kv_bytes_per_step": wl.kv_bytes(),
         "l2": ("inputs larger than L2 (KV %d MB > 126 MB L2), no flush"
                % (wl.kv_bytes() // 10**6)) if wl.kv_bytes() > L2_BYTES else
@@ -428,11 +437,25 @@ def main():
                                        v_scale=v_scale, max_context_len=max_ctx, out=out,
                                        workspace=ws, num_splits=splits, err_flag=err)
 
+    # one launch per step (append fused into the decode kernel) unless asked
+    # otherwise; the shared-prefix cascade and fp32 caches take the two calls
+    fused = not prefix_len and not args.unfused and wl.cache_dtype != "f32"
+
+    def attend_append(qq, kk, vv, ss, btt, cll):
+        pkv.paged_attention_decode_append(qq, kk, vv, ss, k_cache, v_cache, btt, cll,
+                                          softmax_scale=wl.softmax_scale, k_scale=k_scale,
+                                          v_scale=v_scale, max_context_len=max_ctx, out=out,
+                                          workspace=ws, num_splits=splits, err_flag=err)
+
     def step(ev_pair=None):
-        pkv.kv_cache_append(nk, nv, ns, k_cache, v_cache, k_scale, v_scale, err_flag=err)
+        if not fused:
+            pkv.kv_cache_append(nk, nv, ns, k_cache, v_cache, k_scale, v_scale, err_flag=err)
         if ev_pair is not None:
             ev_pair[0].record()
-        attend(q, bt, cl)
+        if fused:
+            attend_append(q, nk, nv, ns, bt, cl)
+        else:
+            attend(q, bt, cl)
         if ev_pair is not None:
             ev_pair[1].record()
 
@@ -526,8 +549,12 @@ def main():
 
         def e2e_step():
             dbuf.copy_(hbuf, non_blocking=True)
-            pkv.kv_cache_append(dk, dv, dsl, k_cache, v_cache, k_scale, v_scale, err_flag=err)
-            attend(dq, dbt, dcl)
+            if fused:
+                attend_append(dq, dk, dv, dsl, dbt, dcl)
+            else:
+                pkv.kv_cache_append(dk, dv, dsl, k_cache, v_cache, k_scale, v_scale,
+                                    err_flag=err)
+                attend(dq, dbt, dcl)
             hout.copy_(out, non_blocking=True)
 
         for _ in range(W):
@@ -557,7 +584,8 @@ def main():
     if rank == 0:
         ms_per_step = max_ms / K
         layers = LAYERS.get(wl.name, 1)
-        launches_per_step = (4 if prefix_len else 2 + (1 if splits > 1 else 0))
+        launches_per_step = (4 if prefix_len else
+                             (1 if fused else 2) + (1 if splits > 1 else 0))
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5),
@@ -575,6 +603,8 @@ def main():
                          "traffic": traffic,
                          "kernel": ("pkv_paged_attention_decode_shared_prefix (prefix pass + "
                                     "suffix decode + merge; logical KV bytes)" if prefix_len else
+                                    "pkv_paged_attention_decode_append (append + decode + "
+                                    "split merge)" if fused else
                                     "pkv_paged_attention_decode (decode + split merge)"),
                          "peak_source": f"{peak_kind} (hbm_gbs)",
                          "decode_ms_mean": round(decode_ms, 5),

@@ -157,6 +157,42 @@ int pkv_paged_attention_decode(void* out, const void* q, pkv_dtype q_dt, const v
                                int num_splits, int* err_flag, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_decode_append - one decode step in one call: each
+ * sequence's new token is appended ([yunthe], KV-cache overhead section: every
+ * generated token's K/V goes into the cache; §4 of [mlqm] for the quantised
+ * rows) and the sequence then attends over its context_lens tokens, new token
+ * included.  The result, cache contents included, is that of
+ * pkv_kv_cache_append(k, v, slot_mapping, num_seqs tokens) followed by
+ * pkv_paged_attention_decode, provided slot_mapping[s] is the slot the block
+ * table gives position context_lens[s] - 1 of sequence s.  The CTA that
+ * attends that position writes the token's rows of its KV head first, so no
+ * separate append launch is needed.
+ *
+ * Arguments as for pkv_paged_attention_decode, plus:
+ *   k, v          device bf16 [num_seqs][num_kv_heads][head_dim], contiguous,
+ *                 16-byte aligned: the new token of each sequence.
+ *   slot_mapping  device int64 [num_seqs], 8-byte aligned.  A negative slot
+ *                 writes nothing.  A slot that is not the one of position
+ *                 context_lens[s] - 1 (or outside the pool) writes nothing and
+ *                 sets PKV_FLAG_BAD_SLOT.
+ *   in_dt         PKV_BF16 (k, v and q).
+ *   k_cache, v_cache, k_scale, v_scale  written (the new rows and scales).
+ * Supported: cache_dt PKV_BF16, PKV_I8 or PKV_FP8 (PKV_F32:
+ * PKV_ERR_UNSUPPORTED; use the two calls).
+ */
+int pkv_paged_attention_decode_append(void* out, const void* q, const void* k, const void* v,
+                                      const int64_t* slot_mapping, pkv_dtype in_dt,
+                                      void* k_cache, void* v_cache, pkv_dtype cache_dt,
+                                      float* k_scale, float* v_scale,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int max_context_len,
+                                      int num_seqs, int num_q_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int num_blocks,
+                                      float softmax_scale, void* workspace,
+                                      size_t workspace_bytes, int num_splits, int* err_flag,
+                                      pkv_stream_t stream);
+
+/*
  * pkv_paged_attention_decode_shared_prefix - pkv_paged_attention_decode for a
  * batch whose sequences all begin with the same `prefix_len` tokens stored in
  * the same physical blocks (prefix caching: "生产级 LLM 推理的 KV 缓存优化"

@@ -32,6 +32,9 @@ SIGNATURES = {
     "pkv_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "pkv_paged_attention_decode": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i, _vp, _i,
                                         _i, _i, _i, _i, _i, _i, _f, _vp, _sz, _i, _vp, _vp]),
+    "pkv_paged_attention_decode_append": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp,
+                                               _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                               _f, _vp, _sz, _i, _vp, _vp]),
     "pkv_paged_attention_decode_noalloc": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i,
                                                 _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                                                 _vp]),

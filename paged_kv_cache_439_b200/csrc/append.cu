@@ -96,20 +96,8 @@ __global__ void __launch_bounds__(kAppendThreads)
   float x[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) x[e] = to_f32(src[e]);
-  float amax = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = (amax > 0.f) ? __fdiv_rn(127.0f, amax) : 1.0f;
-  uint32_t packed = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    float r = rintf(__fmul_rn(x[e], scale));
-    r = fminf(fmaxf(r, -128.f), 127.f);
-    const int qv = (amax > 0.f) ? (int)r : 0;
-    packed |= (uint32_t)(qv & 0xff) << (8 * e);
-  }
+  float scale;
+  const uint32_t packed = quant_row_int8<E>(x, &scale);
   const long long blk = slot / block_size;
   const int off = (int)(slot % block_size);
   int8_t* dst = (is_v ? v_cache : k_cache) + ((size_t)slot * num_kv_heads + h) * HD + lane * E;
@@ -152,18 +140,8 @@ __global__ void __launch_bounds__(kAppendThreads)
   float x[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) x[e] = to_f32(src[e]);
-  float amax = 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = (amax > 0.f) ? __fdiv_rn(448.0f, amax) : 1.0f;
-  uint32_t packed = 0;
-  if (amax > 0.f) {
-#pragma unroll
-    for (int e = 0; e < E; e += 2)
-      packed |= f32x2_to_e4m3x2(__fmul_rn(x[e], scale), __fmul_rn(x[e + 1], scale)) << (8 * e);
-  }
+  float scale;
+  const uint32_t packed = quant_row_fp8<E>(x, &scale);
   const long long blk = slot / block_size;
   const int off = (int)(slot % block_size);
   uint8_t* dst = (is_v ? v_cache : k_cache) + ((size_t)slot * num_kv_heads + h) * HD + lane * E;

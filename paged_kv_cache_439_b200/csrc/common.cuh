@@ -169,6 +169,53 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Row quantisers of the cache append rule, for one warp per (token, head) row:
+// lane l holds the row's elements E*l .. E*l+E-1 (E = head_dim / 32) as fp32.
+// Both return the lane's codes packed into the low 8*E bits (first element in
+// the lowest byte) and leave the row's scale in *scale.
+// INT8 (the mlqm page, §4 quantize_tensor): scale = 127 / max|x| over the row,
+// code = clamp(rint(x * scale), -128, 127), division and product correctly
+// rounded and unfused; an all-zero row gives codes 0 and scale 1.
+template <int E>
+__device__ __forceinline__ uint32_t quant_row_int8(const float (&x)[E], float* scale) {
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float s = (amax > 0.f) ? __fdiv_rn(127.0f, amax) : 1.0f;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    float r = rintf(__fmul_rn(x[e], s));
+    r = fminf(fmaxf(r, -128.f), 127.f);
+    const int qv = (amax > 0.f) ? (int)r : 0;
+    packed |= (uint32_t)(qv & 0xff) << (8 * e);
+  }
+  *scale = s;
+  return packed;
+}
+
+// FP8 (E4M3) form of the same rule: scale = 448 / max|x|, codes E4M3(x * scale)
+// rounded to nearest even and saturated; an all-zero row gives codes 0, scale 1.
+template <int E>
+__device__ __forceinline__ uint32_t quant_row_fp8(const float (&x)[E], float* scale) {
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const float s = (amax > 0.f) ? __fdiv_rn(448.0f, amax) : 1.0f;
+  uint32_t packed = 0;
+  if (amax > 0.f) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2)
+      packed |= f32x2_to_e4m3x2(__fmul_rn(x[e], s), __fmul_rn(x[e + 1], s)) << (8 * e);
+  }
+  *scale = s;
+  return packed;
+}
+
 __device__ __forceinline__ float fast_rcp(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));

@@ -31,6 +31,7 @@ namespace pkv {
 
 struct CtaSetup {
   int seq, kvh, split;
+  int ctx;             // the sequence's (clamped) context length
   int t_begin, t_end;  // token range of this CTA
   int blk0;            // first logical block in s_phys
   bool active;
@@ -63,6 +64,7 @@ __device__ __forceinline__ CtaSetup cta_setup(const DecodeParams& p, int* s_phys
   const bool report = (c.kvh == 0 && c.split == 0 && threadIdx.x == 0);
   const int ctx = effective_ctx(p, c.seq, report);
   c.t_begin = p.t_start + c.split * p.chunk;
+  c.ctx = ctx;
   c.t_end = min(ctx, c.t_begin + p.chunk);
   c.active = c.t_begin < c.t_end;
   c.blk0 = c.t_begin >> p.log2_bs;
@@ -80,6 +82,100 @@ __device__ __forceinline__ CtaSetup cta_setup(const DecodeParams& p, int* s_phys
   }
   __syncthreads();
   return c;
+}
+
+// Cache formats of the mma engine.
+constexpr int kQuantNone = 0;  // bf16 values
+constexpr int kQuantI8 = 1;    // int8 codes, fp32 scale per token per head
+constexpr int kQuantFp8 = 2;   // E4M3 codes, fp32 scale per token per head
+
+// Fused append (pkv_paged_attention_decode_append), in two parts.
+//
+// Prefetch, in every warp before the CTA's first barrier: each lane loads its
+// share of the sequence's new K and V rows of this KV head (bf16 rows: lane l
+// holds 16-byte chunk l of K, then of V; one-byte caches: lane l holds
+// elements E*l .. E*l+E-1 of K in .x/.y and of V in .z/.w, E = head_dim / 32)
+// and the token's slot, so their latency overlaps the CTA set-up.
+template <int HD, int QM>
+__device__ __forceinline__ uint4 fused_prefetch(const DecodeParams& p, long long* slot) {
+  uint4 r = make_uint4(0u, 0u, 0u, 0u);
+  *slot = -1;
+  if (p.new_k == nullptr) return r;
+  const int lane = threadIdx.x % kWarp;
+  const size_t base = ((size_t)blockIdx.y * p.num_kv_heads + blockIdx.x) * HD;
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.new_k) + base;
+  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.new_v) + base;
+  *slot = p.slot_mapping[blockIdx.y];
+  if constexpr (QM == kQuantNone) {
+    constexpr int V = HD / 8;  // 16-byte chunks of a bf16 row
+    if (lane < 2 * V) r = reinterpret_cast<const uint4*>(lane < V ? k : v)[lane % V];
+  } else if constexpr (HD / kWarp == 4) {
+    const uint2 a = reinterpret_cast<const uint2*>(k)[lane];
+    const uint2 b = reinterpret_cast<const uint2*>(v)[lane];
+    r = make_uint4(a.x, a.y, b.x, b.y);
+  } else {
+    r.x = reinterpret_cast<const uint32_t*>(k)[lane];
+    r.z = reinterpret_cast<const uint32_t*>(v)[lane];
+  }
+  return r;
+}
+
+// Commit, after the set-up: the warp that will read the 16-token tile holding
+// position ctx - 1 (tile i of the CTA belongs to warp i % NWARPS) writes the
+// token's K and V rows into slot_mapping[seq], quantised for one-byte caches
+// with the append kernels' own row rule, then syncs the warp, so that its
+// later cp.async reads of that position see the rows.  No other CTA reads the
+// position.  The slot must be the one the block table gives position ctx - 1;
+// otherwise nothing is written and PKV_FLAG_BAD_SLOT is set.  A negative slot
+// writes nothing.
+template <int HD, int QM, int NWARPS>
+__device__ __forceinline__ void fused_commit(const DecodeParams& p, const CtaSetup& c,
+                                             const int* s_phys, uint4 r, long long slot) {
+  if (p.new_k == nullptr || !c.active || c.t_end != c.ctx) return;
+  const int pos = c.ctx - 1;
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  if (warp != ((pos - c.t_begin) >> 4) % NWARPS || slot < 0) return;
+  const int bs = p.block_size;
+  const int b = s_phys[(pos >> p.log2_bs) - c.blk0];
+  if (b < 0 || slot != (long long)b * bs + (pos & (bs - 1))) {
+    if (lane == 0) set_flag(p.err_flag, PKV_FLAG_BAD_SLOT);
+    return;
+  }
+  const size_t row = (size_t)slot * p.num_kv_heads + c.kvh;  // in head_dim units
+  if constexpr (QM == kQuantNone) {
+    constexpr int V = HD / 8;
+    if (lane < 2 * V) {
+      void* cache = const_cast<void*>(lane < V ? p.k_cache : p.v_cache);
+      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(cache) + row * HD)[lane % V] = r;
+    }
+  } else {
+    constexpr int E = HD / kWarp;  // elements per lane
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {  // K, then V
+      const uint32_t w0 = t ? r.z : r.x, w1 = t ? r.w : r.y;
+      float x[E];
+      x[0] = __uint_as_float(w0 << 16);
+      x[1] = __uint_as_float(w0 & 0xFFFF0000u);
+      if constexpr (E == 4) {
+        x[2] = __uint_as_float(w1 << 16);
+        x[3] = __uint_as_float(w1 & 0xFFFF0000u);
+      }
+      float scale;
+      const uint32_t packed =
+          QM == kQuantI8 ? quant_row_int8<E>(x, &scale) : quant_row_fp8<E>(x, &scale);
+      uint8_t* dst = static_cast<uint8_t*>(const_cast<void*>(t ? p.v_cache : p.k_cache)) +
+                     row * HD + lane * E;
+      if constexpr (E == 4)
+        *reinterpret_cast<uint32_t*>(dst) = packed;
+      else
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+      if (lane == 0) {
+        float* sc = const_cast<float*>(t ? p.v_scale : p.k_scale);
+        sc[((size_t)b * p.num_kv_heads + c.kvh) * bs + (pos & (bs - 1))] = scale;
+      }
+    }
+  }
+  __syncwarp();
 }
 
 // Physical block of token t (-1 when masked: past the range or bad block).
@@ -240,10 +336,6 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 #define PKV_I8_STAGES 3
 #endif
 
-// Cache formats of the mma engine.
-constexpr int kQuantNone = 0;  // bf16 values
-constexpr int kQuantI8 = 1;    // int8 codes, fp32 scale per token per head
-constexpr int kQuantFp8 = 2;   // E4M3 codes, fp32 scale per token per head
 
 template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
 struct MmaCfg {
@@ -351,11 +443,14 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   int* s_phys = reinterpret_cast<int*>(smem);
   uint8_t* ring = smem + p.phys_bytes;
 
+  long long new_slot;
+  const uint4 new_rows = fused_prefetch<HD, QM>(p, &new_slot);
   const CtaSetup c = cta_setup(p, s_phys);
   if (!c.active) {
     if (c.split == 0) store_zero<HD>(p, c);
     return;
   }
+  fused_commit<HD, QM, NWARPS>(p, c, s_phys, new_rows, new_slot);  // before any cache read
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int g = lane >> 2, t4 = lane & 3;
   const int G = p.group;

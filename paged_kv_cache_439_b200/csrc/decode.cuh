@@ -34,6 +34,12 @@ struct DecodeParams {
   float scale_log2;  // softmax_scale * log2(e)
   int q_f32;
   int out_f32;
+  // Fused append (pkv_paged_attention_decode_append): sequence s's new token,
+  // written into its slot by the CTA that attends position context_lens[s] - 1
+  // before that CTA reads the cache.  Null for a plain decode.
+  const void* new_k = nullptr;             // [num_seqs][num_kv_heads][head_dim] bf16
+  const void* new_v = nullptr;
+  const int64_t* slot_mapping = nullptr;   // [num_seqs]
 };
 
 // Shared-prefix pass (prefix.cu): slices of the common prefix, all rows at once.

@@ -87,6 +87,27 @@ def test_decode_argument_errors(lib):
     assert _decode(lib, maxb=1024, maxctx=16384, splits=1) == -4
 
 
+def test_fused_decode_append_argument_errors(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, sm=FAKE, idt=1, kc=FAKE, vc=FAKE, cdt=1,
+                 ks=None, vs=None, bt=FAKE, maxb=4, cl=FAKE, maxctx=64, B=2, nq=4, nkv=2, d=128,
+                 bs=16, nb=8, scale=0.125, ws=None, wsb=0, splits=1, err=None)
+        a.update(kw)
+        return lib.pkv_paged_attention_decode_append(
+            a["out"], a["q"], a["k"], a["v"], a["sm"], a["idt"], a["kc"], a["vc"], a["cdt"],
+            a["ks"], a["vs"], a["bt"], a["maxb"], a["cl"], a["maxctx"], a["B"], a["nq"], a["nkv"],
+            a["d"], a["bs"], a["nb"], a["scale"], a["ws"], a["wsb"], a["splits"], a["err"], None)
+    assert call(k=None) == -1
+    assert call(sm=None) == -1
+    assert call(cdt=0, idt=0) == -4                    # fp32 caches: append, then decode
+    assert call(idt=0) == -2                           # new rows must be bf16
+    assert call(k=FAKE + 8) == -7                      # misaligned rows
+    assert call(sm=FAKE + 4) == -7                     # misaligned slot mapping
+    assert call(cdt=2) == -1                           # int8 without scales
+    assert call(nq=6, nkv=4) == -1                     # decode checks apply as well
+    assert call(B=0) == 0
+
+
 def test_append_argument_errors(lib):
     def call(**kw):
         a = dict(k=FAKE, v=FAKE, sm=FAKE, T=4, nkv=2, d=64, idt=1, kc=FAKE, vc=FAKE, cdt=1, nb=4,
