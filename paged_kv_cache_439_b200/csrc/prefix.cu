@@ -163,7 +163,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 
 // One lane per warp polls while the others wait at the warp barrier, so that
 // waiting warps do not flood the shared-memory pipe that the copies and the
-// tensor-memory loads go through.  Every lane gets the verdict.
+// tensor-memory loads go through.  Every lane gets the result.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
   int ok = 1;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1 : 0;
