@@ -268,11 +268,10 @@ def config_dict(wl, args, splits):
         "head_dim": wl.head_dim, "block_size": wl.block_size, "cache_dtype": wl.cache_dtype,
         "num_blocks": wl.num_blocks, "num_splits": splits,
         "shared_prefix_pass": bool(getattr(args, "cascade", False)),
-        "step": ("kv_cache_append (1 new token per sequence) + paged_attention_decode"
-                 if (getattr(args, "cascade", False) or getattr(args, "unfused", False)
-                     or wl.cache_dtype == "f32") else
-                 "paged_attention_decode_append (1 new token per sequence appended inside "
-                 "the decode kernel)"),
+        "step": ("kv_cache_append (1 new token per sequence) + the attention call"
+                 if (getattr(args, "unfused", False) or wl.cache_dtype == "f32") else
+                 "the attention call with the append fused in (1 new token per sequence "
+                 "written inside the decode kernel)"),
         "kv_bytes_per_step": wl.kv_bytes(),
         "l2": ("inputs larger than L2 (KV %d MB > 126 MB L2), no flush"
                % (wl.kv_bytes() // 10**6)) if wl.kv_bytes() > L2_BYTES else
@@ -437,15 +436,21 @@ def main():
                                        v_scale=v_scale, max_context_len=max_ctx, out=out,
                                        workspace=ws, num_splits=splits, err_flag=err)
 
-    # one launch per step (append fused into the decode kernel) unless asked
-    # otherwise; the shared-prefix cascade and fp32 caches take the two calls
-    fused = not prefix_len and not args.unfused and wl.cache_dtype != "f32"
+    # the append fused into the attention call unless asked otherwise (fp32
+    # caches have no fused form)
+    fused = not args.unfused and wl.cache_dtype != "f32"
 
     def attend_append(qq, kk, vv, ss, btt, cll):
-        pkv.paged_attention_decode_append(qq, kk, vv, ss, k_cache, v_cache, btt, cll,
-                                          softmax_scale=wl.softmax_scale, k_scale=k_scale,
-                                          v_scale=v_scale, max_context_len=max_ctx, out=out,
-                                          workspace=ws, num_splits=splits, err_flag=err)
+        if prefix_len:
+            pkv.paged_attention_decode_shared_prefix_append(
+                qq, kk, vv, ss, k_cache, v_cache, btt, cll, prefix_len,
+                softmax_scale=wl.softmax_scale, max_context_len=max_ctx, out=out, workspace=ws,
+                num_splits=splits, err_flag=err)
+        else:
+            pkv.paged_attention_decode_append(qq, kk, vv, ss, k_cache, v_cache, btt, cll,
+                                              softmax_scale=wl.softmax_scale, k_scale=k_scale,
+                                              v_scale=v_scale, max_context_len=max_ctx, out=out,
+                                              workspace=ws, num_splits=splits, err_flag=err)
 
     def step(ev_pair=None):
         if not fused:
@@ -584,8 +589,8 @@ def main():
     if rank == 0:
         ms_per_step = max_ms / K
         layers = LAYERS.get(wl.name, 1)
-        launches_per_step = (4 if prefix_len else
-                             (1 if fused else 2) + (1 if splits > 1 else 0))
+        launches_per_step = ((3 if prefix_len else 1 + (1 if splits > 1 else 0)) +
+                             (0 if fused else 1))
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": round(ms_per_step, 5),
@@ -601,8 +606,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic,
-                         "kernel": ("pkv_paged_attention_decode_shared_prefix (prefix pass + "
-                                    "suffix decode + merge; logical KV bytes)" if prefix_len else
+                         "kernel": (("pkv_paged_attention_decode_shared_prefix" +
+                                     ("_append" if fused else "") +
+                                     " (prefix pass + suffix decode + merge; logical KV bytes)")
+                                    if prefix_len else
                                     "pkv_paged_attention_decode_append (append + decode + "
                                     "split merge)" if fused else
                                     "pkv_paged_attention_decode (decode + split merge)"),

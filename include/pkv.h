@@ -225,6 +225,28 @@ int pkv_paged_attention_decode_shared_prefix(
     int* err_flag, pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_decode_shared_prefix_append - the shared-prefix decode
+ * with each sequence's new token appended in the same call, by the suffix
+ * decode kernel (as in pkv_paged_attention_decode_append).  The result, cache
+ * included, is that of pkv_kv_cache_append followed by
+ * pkv_paged_attention_decode_shared_prefix, provided slot_mapping[s] is the
+ * slot of position context_lens[s] - 1 and that position lies past the shared
+ * prefix (>= prefix_len); a token inside the shared blocks is not written and
+ * sets PKV_FLAG_BAD_SLOT (shared blocks are not written through this call).
+ * Arguments as for pkv_paged_attention_decode_shared_prefix, plus k, v
+ * (device bf16 [num_seqs][num_kv_heads][head_dim], 16-byte aligned) and
+ * slot_mapping (device int64 [num_seqs], 8-byte aligned; negative: nothing
+ * written).  Supported: cache_dt PKV_BF16, in_dt PKV_BF16.
+ */
+int pkv_paged_attention_decode_shared_prefix_append(
+    void* out, const void* q, const void* k, const void* v, const int64_t* slot_mapping,
+    pkv_dtype in_dt, void* k_cache, void* v_cache, pkv_dtype cache_dt,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+    int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int num_blocks, float softmax_scale, int prefix_len, void* workspace,
+    size_t workspace_bytes, int num_splits, int* err_flag, pkv_stream_t stream);
+
+/*
  * pkv_copy - device-to-device copy of `bytes` bytes (a multiple of 16) with a
  * streaming kernel; used to measure the attainable HBM bandwidth in the same
  * process as the attention kernels.  Not part of the attention path.

@@ -35,6 +35,10 @@ SIGNATURES = {
     "pkv_paged_attention_decode_append": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _vp,
                                                _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i,
                                                _f, _vp, _sz, _i, _vp, _vp]),
+    "pkv_paged_attention_decode_shared_prefix_append": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _vp,
+                                                             _vp, _i, _vp, _i, _vp, _i, _i,
+                                                             _i, _i, _i, _i, _i, _f, _i, _vp,
+                                                             _sz, _i, _vp, _vp]),
     "pkv_paged_attention_decode_noalloc": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _i,
                                                 _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                                                 _vp]),

@@ -241,6 +241,44 @@ def paged_attention_decode_shared_prefix(q: torch.Tensor, k_cache: torch.Tensor,
     return out
 
 
+def paged_attention_decode_shared_prefix_append(
+        q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+        k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+        context_lens: torch.Tensor, prefix_len: int, softmax_scale: Optional[float] = None,
+        max_context_len: Optional[int] = None, out: Optional[torch.Tensor] = None,
+        workspace: Optional[torch.Tensor] = None, num_splits: int = 0,
+        err_flag: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """paged_attention_decode_shared_prefix with each sequence's new token k, v
+    [B, n_kv, d] appended at slot_mapping [B] in the same call (the token's
+    position context_lens[s] - 1 must lie past the shared prefix)."""
+    B, nq, d = q.shape
+    nb, bs, nkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d)
+    maxb = block_tables.shape[1]
+    if max_context_len is None:
+        max_context_len = maxb * bs
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        need = shared_prefix_workspace_size(B, nq, nkv, d, max_context_len, prefix_len,
+                                            k_cache.dtype, num_splits)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if k.shape != (B, nkv, d) or v.shape != (B, nkv, d) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k and v must be [num_seqs, num_kv_heads, head_dim] in q's dtype")
+    rc = N.lib().pkv_paged_attention_decode_shared_prefix_append(
+        _ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(slot_mapping), _dt(q), _ptr(k_cache),
+        _ptr(v_cache), _dt(k_cache), _ptr(block_tables), maxb, _ptr(context_lens),
+        max_context_len, B, nq, nkv, d, bs, nb, float(softmax_scale), prefix_len,
+        _ptr(workspace), workspace.numel(), num_splits, _ptr(err_flag), _stream(stream))
+    N.check(rc, "pkv_paged_attention_decode_shared_prefix_append")
+    return out
+
+
 def copy(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
     """Streaming device copy (HBM bandwidth probe)."""
     nbytes = src.numel() * src.element_size()

@@ -373,20 +373,27 @@ size_t pkv_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_k
       .ws;
 }
 
-int pkv_paged_attention_decode_shared_prefix(
+}  // extern "C"
+
+namespace {
+
+// Shared-prefix decode, optionally with the fused append of each sequence's new
+// token (new_k, new_v, slot_mapping non-null; done by the suffix decode kernel).
+int shared_prefix_impl(
     void* out, const void* q, pkv_dtype q_dt, const void* k_cache, const void* v_cache,
     pkv_dtype cache_dt, const float* k_scale, const float* v_scale, const int32_t* block_tables,
     int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
     int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
     float softmax_scale, int prefix_len, void* workspace, size_t workspace_bytes, int num_splits,
-    int* err_flag, pkv_stream_t stream) {
+    int* err_flag, pkv_stream_t stream, const void* new_k, const void* new_v,
+    const int64_t* slot_mapping) {
   if (prefix_len < 0) return PKV_ERR_ARG;
   if (prefix_len == 0)
-    return pkv_paged_attention_decode(out, q, q_dt, k_cache, v_cache, cache_dt, k_scale, v_scale,
-                                      block_tables, max_blocks_per_seq, context_lens,
-                                      max_context_len, num_seqs, num_q_heads, num_kv_heads,
-                                      head_dim, block_size, num_blocks, softmax_scale, workspace,
-                                      workspace_bytes, num_splits, err_flag, stream);
+    return decode_impl(out, q, q_dt, k_cache, v_cache, cache_dt, k_scale, v_scale, block_tables,
+                       max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, softmax_scale, workspace,
+                       workspace_bytes, num_splits, err_flag, stream, new_k, new_v,
+                       slot_mapping);
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
       max_blocks_per_seq <= 0 || max_context_len < 0 || num_splits < 0)
     return PKV_ERR_ARG;
@@ -457,11 +464,51 @@ int pkv_paged_attention_decode_shared_prefix(
   pp.rows = num_seqs * group;
   pp.phys_bytes = round_up((pl.pchunk / block_size + 2) * 4, 128);
 
+  p.new_k = new_k;
+  p.new_v = new_v;
+  p.slot_mapping = slot_mapping;
+
   cudaStream_t st = (cudaStream_t)stream;
   if (pkv::launch_prefix(p, pp, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   if (pkv::launch_merge(p, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_attention_decode_shared_prefix(
+    void* out, const void* q, pkv_dtype q_dt, const void* k_cache, const void* v_cache,
+    pkv_dtype cache_dt, const float* k_scale, const float* v_scale, const int32_t* block_tables,
+    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+    int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+    float softmax_scale, int prefix_len, void* workspace, size_t workspace_bytes, int num_splits,
+    int* err_flag, pkv_stream_t stream) {
+  return shared_prefix_impl(out, q, q_dt, k_cache, v_cache, cache_dt, k_scale, v_scale,
+                            block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                            num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            num_blocks, softmax_scale, prefix_len, workspace, workspace_bytes,
+                            num_splits, err_flag, stream, nullptr, nullptr, nullptr);
+}
+
+int pkv_paged_attention_decode_shared_prefix_append(
+    void* out, const void* q, const void* k, const void* v, const int64_t* slot_mapping,
+    pkv_dtype in_dt, void* k_cache, void* v_cache, pkv_dtype cache_dt,
+    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+    int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+    int block_size, int num_blocks, float softmax_scale, int prefix_len, void* workspace,
+    size_t workspace_bytes, int num_splits, int* err_flag, pkv_stream_t stream) {
+  if (!k || !v || !slot_mapping) return PKV_ERR_ARG;
+  if (cache_dt != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (in_dt != PKV_BF16) return PKV_ERR_DTYPE;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(slot_mapping, 8)) return PKV_ERR_ALIGN;
+  return shared_prefix_impl(out, q, in_dt, k_cache, v_cache, cache_dt, nullptr, nullptr,
+                            block_tables, max_blocks_per_seq, context_lens, max_context_len,
+                            num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            num_blocks, softmax_scale, prefix_len, workspace, workspace_bytes,
+                            num_splits, err_flag, stream, k, v, slot_mapping);
 }
 
 int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream) {

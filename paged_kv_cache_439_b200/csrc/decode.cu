@@ -447,7 +447,14 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   const uint4 new_rows = fused_prefetch<HD, QM>(p, &new_slot);
   const CtaSetup c = cta_setup(p, s_phys);
   if (!c.active) {
-    if (c.split == 0) store_zero<HD>(p, c);
+    if (c.split == 0) {
+      // a new token inside a shared prefix (positions below t_start) has no
+      // CTA of this kernel to write it: report it instead
+      if (p.new_k != nullptr && new_slot >= 0 && c.ctx >= 1 && c.ctx - 1 < p.t_start &&
+          threadIdx.x == 0)
+        set_flag(p.err_flag, PKV_FLAG_BAD_SLOT);
+      store_zero<HD>(p, c);
+    }
     return;
   }
   fused_commit<HD, QM, NWARPS>(p, c, s_phys, new_rows, new_slot);  // before any cache read

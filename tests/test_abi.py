@@ -108,6 +108,26 @@ def test_fused_decode_append_argument_errors(lib):
     assert call(B=0) == 0
 
 
+def test_fused_shared_prefix_argument_errors(lib):
+    def call(**kw):
+        a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, sm=FAKE, idt=1, kc=FAKE, vc=FAKE, cdt=1,
+                 bt=FAKE, maxb=16, cl=FAKE, maxctx=200, B=2, nq=4, nkv=2, d=128, bs=16, nb=32,
+                 scale=0.125, prefix=128, ws=None, wsb=0, splits=1, err=None)
+        a.update(kw)
+        return lib.pkv_paged_attention_decode_shared_prefix_append(
+            a["out"], a["q"], a["k"], a["v"], a["sm"], a["idt"], a["kc"], a["vc"], a["cdt"],
+            a["bt"], a["maxb"], a["cl"], a["maxctx"], a["B"], a["nq"], a["nkv"], a["d"],
+            a["bs"], a["nb"], a["scale"], a["prefix"], a["ws"], a["wsb"], a["splits"], a["err"],
+            None)
+    assert call(v=None) == -1
+    assert call(cdt=2) == -4                           # bf16 caches only
+    assert call(idt=0) == -2
+    assert call(sm=FAKE + 4) == -7
+    assert call(prefix=-16) == -1
+    assert call(prefix=24) == -1                       # not a multiple of block_size
+    assert call(B=0) == 0
+
+
 def test_append_argument_errors(lib):
     def call(**kw):
         a = dict(k=FAKE, v=FAKE, sm=FAKE, T=4, nkv=2, d=64, idt=1, kc=FAKE, vc=FAKE, cdt=1, nb=4,

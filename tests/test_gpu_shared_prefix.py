@@ -11,7 +11,7 @@ import torch
 import paged_kv_cache_439_b200 as pkv
 from paged_kv_cache_439_b200.workloads import make_custom, make_workload
 
-from pkv_testlib import GpuCache, OracleCache, assert_close, tol_for
+from pkv_testlib import GpuCache, OracleCache, assert_close, bits, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -133,3 +133,62 @@ def test_repeated_calls_never_stall():
             max_context_len=wl.max_context_len, num_splits=it % 3, err_flag=g.err)
     torch.cuda.synchronize()
     assert g.flags() == 0
+
+
+def _cascade_append(g, wl, prefix_len, slots=None, **kw):
+    dev = g.device
+    return pkv.paged_attention_decode_shared_prefix_append(
+        wl.q.to(dev), wl.new_k.to(dev), wl.new_v.to(dev),
+        (wl.new_slots if slots is None else slots).to(dev), g.k, g.v,
+        wl.block_tables.to(dev), wl.context_lens.to(dev), prefix_len,
+        softmax_scale=wl.softmax_scale, max_context_len=int(wl.context_lens.max()),
+        err_flag=g.err, **kw)
+
+
+@pytest.mark.parametrize("bs", [16, 256])
+def test_cascade_with_fused_append_equals_two_calls(bs):
+    prefix = 256 if bs == 256 else 512
+    lens = [prefix + x for x in (1, 17, 100, 5, 64, 300)]
+    wl = make_custom(f"sp-fused-{bs}", lens, 8, 2, 128, bs, "bf16", seed=37, shared_prefix=prefix)
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1, 3):
+        two = GpuCache(wl)
+        two.append(wl.prefill_k, wl.prefill_v, wl.prefill_slots)
+        two.append(wl.new_k, wl.new_v, wl.new_slots)
+        out_two = _cascade(two, wl, prefix, num_splits=splits)
+        one = GpuCache(wl)
+        one.append(wl.prefill_k, wl.prefill_v, wl.prefill_slots)
+        out_one = _cascade_append(one, wl, prefix, num_splits=splits)
+        torch.cuda.synchronize()
+        assert one.flags() == 0 and two.flags() == 0
+        assert np.array_equal(bits(one.k), bits(two.k)) and np.array_equal(bits(one.v), bits(two.v))
+        assert np.array_equal(bits(out_one), bits(out_two)), f"splits={splits}"
+        assert_close(out_one, ref, tol_for(wl), f"{wl.name} splits={splits}")
+
+
+def test_cascade_append_refuses_a_token_inside_the_shared_prefix():
+    wl = make_custom("sp-fused-in", [200, 150], 4, 1, 128, 16, "bf16", seed=38, shared_prefix=128)
+    g = GpuCache(wl)
+    g.append(wl.prefill_k, wl.prefill_v, wl.prefill_slots)
+    before = bits(g.k).copy()
+    cl = torch.tensor([100, 150], dtype=torch.int32)   # sequence 0's position 99 is shared
+    slots = wl.new_slots.clone()
+    slots[1] = -1
+    dev = g.device
+    pkv.paged_attention_decode_shared_prefix_append(
+        wl.q.to(dev), wl.new_k.to(dev), wl.new_v.to(dev), slots.to(dev), g.k, g.v,
+        wl.block_tables.to(dev), cl.to(dev), 128, softmax_scale=wl.softmax_scale,
+        max_context_len=150, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert g.flags() & pkv.PKV_FLAG_BAD_SLOT
+    assert np.array_equal(bits(g.k), before)
+
+
+def test_full_shared_prefix_workload_fused_append():
+    wl = make_workload("shared-prefix")
+    g = GpuCache(wl)
+    g.append(wl.prefill_k, wl.prefill_v, wl.prefill_slots)
+    out = _cascade_append(g, wl, 4096)
+    torch.cuda.synchronize()
+    assert g.flags() == 0
+    assert_close(out, OracleCache(wl).fill().decode(), tol_for(wl), "shared-prefix fused")
