@@ -18,16 +18,30 @@
  *          the physical block of logical block j ([yunthe], PagedAttention
  *          section, the block_table example; [mlqm] §2 BlockTable).
  *
+ * Calls:
+ *   append           pkv_kv_cache_append (bf16/fp32 copy, INT8/FP8 quantising)
+ *   decode           pkv_paged_attention_decode, pkv_decode_num_splits,
+ *                    pkv_workspace_size, pkv_paged_attention_decode_noalloc
+ *   one-launch step  pkv_paged_attention_decode_append (append inside decode)
+ *   shared prefix    pkv_paged_attention_decode_shared_prefix[_append],
+ *                    pkv_shared_prefix_workspace_size
+ *   block manager    pkv_bm_* (host bookkeeping: blocks, ref counts, fork,
+ *                    copy-on-write, swap), pkv_copy_blocks (block copies)
+ *   misc             pkv_copy, pkv_strerror, pkv_version
+ *
  * Conventions shared by every call:
- *   - The caller allocates and owns every buffer; the library keeps no state
- *     between calls, allocates nothing and never synchronises.
+ *   - The caller allocates and owns every device buffer; the GPU calls keep no
+ *     state between calls, allocate nothing and never synchronise.  (Two
+ *     exceptions, each described at its call: the host block manager objects
+ *     of pkv_bm_create, and the fixed device scratch behind
+ *     pkv_paged_attention_decode_noalloc.)
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and targets the current CUDA device.
  *   - Argument errors return a negative pkv_status before anything is launched.
  *   - Data errors found on the device (bad block id, bad slot, context length
  *     out of range) are OR-ed as PKV_FLAG_* bits into *err_flag (a device int,
  *     may be NULL); the offending token/row is skipped, the kernel never traps.
- *   - Device pointers must be 16-byte aligned.
+ *   - Device pointers must be 16-byte aligned unless a call states otherwise.
  */
 #ifndef PKV_H
 #define PKV_H
