@@ -24,26 +24,17 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int s
                : "memory");
 }
 
-// cp_async_16 whose destination address is computed from `dep` inside the asm
-// block, so the copy cannot issue before the instructions producing `dep` have
-// their inputs (used to refill a stage only after every ldmatrix that read it
-// has returned its data).
-__device__ __forceinline__ void cp_async_16_after(uint32_t dst, const void* src, int src_bytes,
-                                                  uint32_t dep) {
-  asm volatile(
-      "{\n .reg .b32 z;\n and.b32 z, %3, 0;\n add.u32 z, z, %0;\n"
-      " cp.async.cg.shared.global [z], [%1], 16, %2;\n}\n" ::"r"(dst),
-      "l"(src), "r"(src_bytes), "r"(dep)
-      : "memory");
-}
-
-__device__ __forceinline__ void cp_async_4_after(uint32_t dst, const void* src, int src_bytes,
-                                                 uint32_t dep) {
-  asm volatile(
-      "{\n .reg .b32 z;\n and.b32 z, %3, 0;\n add.u32 z, z, %0;\n"
-      " cp.async.ca.shared.global [z], [%1], 4, %2;\n}\n" ::"r"(dst),
-      "l"(src), "r"(src_bytes), "r"(dep)
-      : "memory");
+// Returns `addr`, computed from `dep` inside an asm block: a copy whose
+// destination is derived from the result cannot issue before the instructions
+// producing `dep` have their inputs (used to refill a stage only after every
+// ldmatrix that read it has returned its data).  Applied once to a stage's
+// base address, it orders every copy into that stage.
+__device__ __forceinline__ uint32_t after_dep(uint32_t addr, uint32_t dep) {
+  uint32_t r;
+  asm volatile("{\n .reg .b32 z;\n and.b32 z, %2, 0;\n add.u32 %0, z, %1;\n}\n"
+               : "=r"(r)
+               : "r"(addr), "r"(dep));
+  return r;
 }
 
 __device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, int src_bytes) {

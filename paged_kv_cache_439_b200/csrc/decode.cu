@@ -353,11 +353,12 @@ struct MmaCfg {
   static_assert(CH == 4 || CH == 8 || CH == 16, "rows of 64, 128 or 256 bytes");
 };
 
-// Issues the copies of one 16-token tile (K, V and, for INT8, the 16 per-token
-// scales) into a stage, as one commit group.  Full tiles inside one block take
-// the fast path: one block-table lookup and per-lane offsets fixed for the
-// whole kernel.  Rows outside the sequence or in a bad block are zero-filled.
-// With AFTER, every copy waits for `dep` (see cp_async_16_after).
+// Issues the copies of one 16-token tile (K, V and, for one-byte caches, the
+// 16 per-token scales of each) into a stage, as one commit group.  Full tiles
+// inside one block take the fast path: one block-table lookup, one 64-bit base
+// per lane and fixed per-lane offsets.  Rows outside the sequence or in a bad
+// block are zero-filled.  With AFTER, the stage address is derived from `dep`
+// (see after_dep), so no copy overtakes the reads of the stage it overwrites.
 template <class Cfg, bool AFTER>
 __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup& c,
                                            const int* s_phys, int tile_t0, uint32_t k_st,
@@ -368,21 +369,32 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
   const uint8_t* vb = static_cast<const uint8_t*>(p.v_cache);
   const size_t tok_stride = (size_t)p.num_kv_heads * Cfg::ROWB;
   const int bs = p.block_size;
+  if constexpr (AFTER) {
+    k_st = after_dep(k_st, dep);
+    v_st = after_dep(v_st, dep);
+    if constexpr (Cfg::ELEM == 1) sc_st = after_dep(sc_st, dep);
+  }
+  // scale row of this lane: lanes 0-15 copy K scales, 16-31 V scales
+  const int srow = lane & 15;
+  const float* ssrc = (lane < 16) ? p.k_scale : p.v_scale;
   if (bs >= 16 && tile_t0 + 16 <= c.t_end) {
     const int phys = s_phys[(tile_t0 >> p.log2_bs) - c.blk0];
     const int n = phys >= 0 ? 16 : 0;
-    const size_t base =
-        phys >= 0 ? ((size_t)phys * bs + (tile_t0 & (bs - 1))) * tok_stride + lane_goff : 0;
+    const int in_blk = tile_t0 & (bs - 1);
+    // a bad block reads nothing (n = 0); its addresses stay inside the cache
+    const size_t base = phys >= 0 ? ((size_t)phys * bs + in_blk) * tok_stride + lane_goff : 0;
+    const size_t step = (size_t)Cfg::RSTEP * tok_stride;
+    const uint8_t* kp = kb + base;
+    const uint8_t* vp = vb + base;
 #pragma unroll
     for (int i = 0; i < Cfg::PER_LANE; ++i) {
-      const size_t off = phys >= 0 ? base + (size_t)i * Cfg::RSTEP * tok_stride : 0;
-      if constexpr (AFTER) {
-        cp_async_16_after(k_st + soff[i], kb + off, n, dep);
-        cp_async_16_after(v_st + soff[i], vb + off, n, dep);
-      } else {
-        cp_async_16(k_st + soff[i], kb + off, n);
-        cp_async_16(v_st + soff[i], vb + off, n);
-      }
+      cp_async_16(k_st + soff[i], kp + (size_t)i * step, n);
+      cp_async_16(v_st + soff[i], vp + (size_t)i * step, n);
+    }
+    if constexpr (Cfg::ELEM == 1) {
+      const size_t soff_g =
+          phys >= 0 ? ((size_t)phys * p.num_kv_heads + c.kvh) * bs + in_blk + srow : 0;
+      cp_async_4(sc_st + 4 * lane, ssrc + soff_g, phys >= 0 ? 4 : 0);
     }
   } else {
     const size_t lane_col = lane_goff - (size_t)lane_row * tok_stride;  // head + chunk offset
@@ -397,38 +409,29 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
         off = ((size_t)phys * bs + (t & (bs - 1))) * tok_stride + lane_col;
         n = 16;
       }
-      if constexpr (AFTER) {
-        cp_async_16_after(k_st + soff[i], kb + off, n, dep);
-        cp_async_16_after(v_st + soff[i], vb + off, n, dep);
-      } else {
-        cp_async_16(k_st + soff[i], kb + off, n);
-        cp_async_16(v_st + soff[i], vb + off, n);
+      cp_async_16(k_st + soff[i], kb + off, n);
+      cp_async_16(v_st + soff[i], vb + off, n);
+    }
+    if constexpr (Cfg::ELEM == 1) {
+      const int t = tile_t0 + srow;
+      const int phys = phys_of(p, c, s_phys, t);
+      size_t off = 0;
+      int n = 0;
+      if (phys >= 0) {
+        off = ((size_t)phys * p.num_kv_heads + c.kvh) * bs + (t & (bs - 1));
+        n = 4;
       }
+      cp_async_4(sc_st + 4 * lane, ssrc + off, n);
     }
-  }
-  if constexpr (Cfg::ELEM == 1) {
-    const int row = lane & 15;
-    const int t = tile_t0 + row;
-    const int phys = phys_of(p, c, s_phys, t);
-    const float* src = (lane < 16) ? p.k_scale : p.v_scale;
-    size_t off = 0;
-    int n = 0;
-    if (phys >= 0) {
-      off = ((size_t)phys * p.num_kv_heads + c.kvh) * bs + (t & (bs - 1));
-      n = 4;
-    }
-    if constexpr (AFTER)
-      cp_async_4_after(sc_st + 4 * lane, src + off, n, dep);
-    else
-      cp_async_4(sc_st + 4 * lane, src + off, n);
   }
   cp_async_commit();
 }
 
-template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
+template <int HD, int QM, int NT, int NWARPS, int NSTAGES, bool MHA>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_mma_kernel(const DecodeParams p) {
   using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
+  static_assert(!MHA || NT == 1, "MHA: one q head per kv head");
   constexpr bool I8 = QM == kQuantI8;
   constexpr bool F8 = QM == kQuantFp8;
   constexpr bool Q8 = I8 || F8;         // one-byte codes with per-token scales
@@ -567,12 +570,14 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       cp_async_commit();
   }
 
-  for (int i = 0; i < my_n; ++i) {
+  const uint32_t ring_last = my_ring + (uint32_t)((NSTAGES - 1) * Cfg::STAGE);
+  uint32_t kS = my_ring;  // stage of tile i
+  int tile_t0 = c.t_begin + warp * 16;
+  for (int i = 0; i < my_n;
+       ++i, tile_t0 += NWARPS * 16, kS = (kS == ring_last) ? my_ring : kS + Cfg::STAGE) {
     cp_async_wait<NSTAGES - 1>();
     __syncwarp();
-    const uint32_t kS = my_ring + (uint32_t)((i % NSTAGES) * Cfg::STAGE);
     const uint32_t vS = kS + Cfg::TILE;
-    const int tile_t0 = c.t_begin + (warp + i * NWARPS) * 16;
 
     // ---- read the stage into registers
     uint32_t kf[KA][4], vf[VA][4];
@@ -604,7 +609,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     {
       const int ii = i + NSTAGES;
       if (ii < my_n)
-        issue_tile<Cfg, true>(p, c, s_phys, c.t_begin + (warp + ii * NWARPS) * 16, kS, vS,
+        issue_tile<Cfg, true>(p, c, s_phys, tile_t0 + NSTAGES * NWARPS * 16, kS, vS,
                               vS + Cfg::TILE, lane, soff, lane_goff, lane_row, dep);
       else
         cp_async_commit();
@@ -691,23 +696,28 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     bool rescale = false;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      float sv[4];
-      sv[0] = va ? ((acc[nt][0] + acc2[nt][0]) - qbias[nt][0]) * fa : -CUDART_INF_F;
-      sv[1] = va ? ((acc[nt][1] + acc2[nt][1]) - qbias[nt][1]) * fa : -CUDART_INF_F;
-      sv[2] = vb ? ((acc[nt][2] + acc2[nt][2]) - qbias[nt][0]) * fb : -CUDART_INF_F;
-      sv[3] = vb ? ((acc[nt][3] + acc2[nt][3]) - qbias[nt][1]) * fb : -CUDART_INF_F;
       float pr[4];
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
-        float mx = fmaxf(sv[jj], sv[jj + 2]);
+        if (MHA && jj == 1) {  // one q head per kv head: column 2*t4 + 1 holds none
+          pr[1] = pr[3] = 0.f;
+          alpha[nt][1] = 1.f;
+          continue;
+        }
+        // scores of head 2*t4 + jj for tokens g (sa) and g + 8 (sb)
+        const float sa =
+            va ? ((acc[nt][jj] + acc2[nt][jj]) - qbias[nt][jj]) * fa : -CUDART_INF_F;
+        const float sb =
+            vb ? ((acc[nt][jj + 2] + acc2[nt][jj + 2]) - qbias[nt][jj]) * fb : -CUDART_INF_F;
+        float mx = fmaxf(sa, sb);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run[nt][jj], mx);
         const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
         const float a = fast_exp2(m_run[nt][jj] - m_use);
-        pr[jj] = fast_exp2(sv[jj] - m_use);
-        pr[jj + 2] = fast_exp2(sv[jj + 2] - m_use);
+        pr[jj] = fast_exp2(sa - m_use);
+        pr[jj + 2] = fast_exp2(sb - m_use);
         l_run[nt][jj] = l_run[nt][jj] * a + pr[jj] + pr[jj + 2];
         m_run[nt][jj] = m_new;
         alpha[nt][jj] = a;
@@ -1131,11 +1141,22 @@ cudaError_t prepare(int smem) {
   return e;
 }
 
-template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
+// Shared memory of one sm_100 SM, and the part the hardware reserves per CTA.
+constexpr int kSmemPerSm = 228 * 1024, kSmemPerCta = 1024;
+// A dynamic shared-memory request above which at most three CTAs fit an SM.
+constexpr int kThreeCtaSmem = kSmemPerSm / 4 - kSmemPerCta + 16;
+
+template <int HD, int QM, int NT, int NWARPS, int NSTAGES, bool MHA>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
-  const int smem = p.phys_bytes + Cfg::BODY;
-  constexpr auto k = decode_mma_kernel<HD, QM, NT, NWARPS, NSTAGES>;
+  int smem = p.phys_bytes + Cfg::BODY;
+  // The one-byte MHA kernels at head_dim 128 fit four CTAs per SM by
+  // registers, the other one-byte kernels three.  Held to three as well, the
+  // FP8 13B workload ran 3% faster (INT8 within 1%), and the split planner's
+  // occupancy figure (taken from the general kernel) stays exact.
+  if constexpr (MHA && QM != kQuantNone && HD == 128)
+    smem = smem > kThreeCtaSmem ? smem : kThreeCtaSmem;
+  constexpr auto k = decode_mma_kernel<HD, QM, NT, NWARPS, NSTAGES, MHA>;
   cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
@@ -1184,7 +1205,7 @@ template <int HD, int QM>
 int mma_occupancy() {
   constexpr int NS = QM != kQuantNone ? PKV_I8_STAGES : PKV_BF16_STAGES;
   using Cfg = MmaCfg<HD, QM, 1, kMW, NS>;
-  return occupancy<decode_mma_kernel<HD, QM, 1, kMW, NS>>(kMW * kWarp,
+  return occupancy<decode_mma_kernel<HD, QM, 1, kMW, NS, false>>(kMW * kWarp,
                                                           kTypicalPhysBytes + Cfg::BODY);
 }
 
@@ -1198,35 +1219,35 @@ int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim) {
   if (cache_dt == PKV_FP8) return head_dim == 128 ? mma_occupancy<128, kQuantFp8>()
                                                   : mma_occupancy<64, kQuantFp8>();
   const int smem = kF32Warps * kF32Stages * 2 * 16 * head_dim * 4 + 16 * head_dim * 4 + 1024;
-  const int n = (228 * 1024) / (smem + 1024);
+  const int n = kSmemPerSm / (smem + kSmemPerCta);
   return n < 1 ? 1 : n;
 }
+
+namespace {
+
+// Picks the q-head tiling: two n-tiles for groups above 8, the MHA form for a
+// group of one, else one n-tile.
+template <int HD, int QM, int NS>
+cudaError_t launch_mma_group(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  if (p.group > 8) return launch_mma<HD, QM, 2, kMW, NS, false>(p, grid, st);
+  if (p.group == 1) return launch_mma<HD, QM, 1, kMW, NS, true>(p, grid, st);
+  return launch_mma<HD, QM, 1, kMW, NS, false>(p, grid, st);
+}
+
+}  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
                           cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.num_seqs, p.num_splits);
-  const bool two = p.group > 8;
-  if (cache_dt == PKV_BF16) {
-    if (head_dim == 128)
-      return two ? launch_mma<128, kQuantNone, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
-                 : launch_mma<128, kQuantNone, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
-    return two ? launch_mma<64, kQuantNone, 2, kMW, PKV_BF16_STAGES>(p, grid, st)
-               : launch_mma<64, kQuantNone, 1, kMW, PKV_BF16_STAGES>(p, grid, st);
-  }
-  if (cache_dt == PKV_I8) {
-    if (head_dim == 128)
-      return two ? launch_mma<128, kQuantI8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-                 : launch_mma<128, kQuantI8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
-    return two ? launch_mma<64, kQuantI8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-               : launch_mma<64, kQuantI8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
-  }
-  if (cache_dt == PKV_FP8) {
-    if (head_dim == 128)
-      return two ? launch_mma<128, kQuantFp8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-                 : launch_mma<128, kQuantFp8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
-    return two ? launch_mma<64, kQuantFp8, 2, kMW, PKV_I8_STAGES>(p, grid, st)
-               : launch_mma<64, kQuantFp8, 1, kMW, PKV_I8_STAGES>(p, grid, st);
-  }
+  if (cache_dt == PKV_BF16)
+    return head_dim == 128 ? launch_mma_group<128, kQuantNone, PKV_BF16_STAGES>(p, grid, st)
+                           : launch_mma_group<64, kQuantNone, PKV_BF16_STAGES>(p, grid, st);
+  if (cache_dt == PKV_I8)
+    return head_dim == 128 ? launch_mma_group<128, kQuantI8, PKV_I8_STAGES>(p, grid, st)
+                           : launch_mma_group<64, kQuantI8, PKV_I8_STAGES>(p, grid, st);
+  if (cache_dt == PKV_FP8)
+    return head_dim == 128 ? launch_mma_group<128, kQuantFp8, PKV_I8_STAGES>(p, grid, st)
+                           : launch_mma_group<64, kQuantFp8, PKV_I8_STAGES>(p, grid, st);
   if (head_dim == 128) return launch_simt<128, kF32Warps, kF32Stages>(p, grid, st);
   return launch_simt<64, kF32Warps, kF32Stages>(p, grid, st);
 }
