@@ -41,7 +41,9 @@
  *   - Data errors found on the device (bad block id, bad slot, context length
  *     out of range) are OR-ed as PKV_FLAG_* bits into *err_flag (a device int,
  *     may be NULL); the offending token/row is skipped, the kernel never traps.
- *   - Device pointers must be 16-byte aligned unless a call states otherwise.
+ *   - Device pointers must be 16-byte aligned unless a call states otherwise;
+ *     int32 arrays (block tables, context lengths) and err_flag need 4 bytes,
+ *     int64 slot arrays 8.  A misaligned pointer returns PKV_ERR_ALIGN.
  */
 #ifndef PKV_H
 #define PKV_H
@@ -67,7 +69,7 @@ typedef enum {
   PKV_ERR_UNSUPPORTED = -4, /* no kernel for this configuration */
   PKV_ERR_WORKSPACE = -5,   /* split-K needs a workspace of pkv_workspace_size() bytes */
   PKV_ERR_CUDA = -6,        /* a CUDA runtime call or launch failed */
-  PKV_ERR_ALIGN = -7,       /* a device pointer is not 16-byte aligned */
+  PKV_ERR_ALIGN = -7,       /* a device pointer is not aligned as its call requires */
   PKV_ERR_SCRATCH_LIMIT = -8, /* split-K scratch would exceed PKV_NOALLOC_SCRATCH_BYTES */
   PKV_ERR_NO_BLOCKS = -9      /* the block pool cannot supply the blocks an operation needs */
 } pkv_status;
@@ -102,11 +104,11 @@ typedef enum {
  *
  *   k, v          device, [num_tokens][num_kv_heads][head_dim], dtype in_dt
  *                 (PKV_F32 or PKV_BF16), contiguous.  Read only.
- *   slot_mapping  device int64 [num_tokens].
+ *   slot_mapping  device int64 [num_tokens], 8-byte aligned.
  *   k_cache, v_cache  device, cache layout above, dtype cache_dt (== in_dt, PKV_I8
  *                 or PKV_FP8).
  *   k_scale, v_scale  device fp32 scale arrays; required iff cache_dt is PKV_I8 or
- *                 PKV_FP8.
+ *                 PKV_FP8 (4-byte alignment suffices for this call).
  *   err_flag      device int or NULL (PKV_FLAG_BAD_SLOT).
  * Two tokens with the same slot race (last writer wins, unspecified).
  */

@@ -161,7 +161,7 @@ const char* pkv_strerror(int status) {
     case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
     case PKV_ERR_WORKSPACE: return "workspace missing or smaller than pkv_workspace_size()";
     case PKV_ERR_CUDA: return "CUDA runtime error";
-    case PKV_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case PKV_ERR_ALIGN: return "device pointer not aligned as the call requires";
     case PKV_ERR_NO_BLOCKS: return "the block pool has too few free blocks";
     case PKV_ERR_SCRATCH_LIMIT:
       return "split-K scratch for this shape exceeds the fixed no-allocation scratch "
@@ -250,7 +250,8 @@ int decode_impl(void* out, const void* q, pkv_dtype q_dt, const void* k_cache,
     return PKV_ERR_DTYPE;
   }
   if ((cache_dt == PKV_I8 || cache_dt == PKV_FP8) && (!k_scale || !v_scale)) return PKV_ERR_ARG;
-  // INT8 scale rows are fetched with bulk copies, which need 16-byte alignment
+  // the header's convention: 16-byte device pointers (the kernels load q, the
+  // cache rows and the workspace 16 bytes at a time), 4-byte int32 arrays
   if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
       !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(block_tables, 4) ||
       !aligned(context_lens, 4) || !aligned(err_flag, 4) || !aligned(workspace, 16))
