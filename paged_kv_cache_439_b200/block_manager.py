@@ -6,13 +6,14 @@ copy kernel.
 from __future__ import annotations
 
 import ctypes
+import math
 from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
 
 from . import _native as N
-from .api import _ptr, _stream
+from .api import _on, _ptr, _stream
 
 
 class BlockManager:
@@ -131,15 +132,39 @@ def copy_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
     """Copies block pairs[i, 0] of the source pool to block pairs[i, 1] of the
     destination pool (K, V and optional scales).  `pairs` is a device int32
     tensor [n, 2]; pools are device tensors or pinned host tensors."""
-    block_bytes = src_k[0].numel() * src_k.element_size()
+    # the library is given one block size and one block count per pool: every
+    # tensor of a pool must agree with them, or a copy would run past its end
+    if dst_v.shape != dst_k.shape or src_v.shape != src_k.shape or dst_k.dim() < 2:
+        raise ValueError("K and V of a pool must have one shape [num_blocks, ...]")
+    block_bytes = _block_bytes(src_k)
+    if _block_bytes(dst_k) != block_bytes:
+        raise ValueError("source and destination blocks differ in size")
+    scales = (dst_k_scale, dst_v_scale, src_k_scale, src_v_scale)
     sbytes = 0
-    if src_k_scale is not None:
-        sbytes = src_k_scale[0].numel() * src_k_scale.element_size()
+    if any(t is not None for t in scales):
+        if any(t is None for t in scales):
+            raise ValueError("give all four scale pools or none")
+        if (dst_v_scale.shape != dst_k_scale.shape or src_v_scale.shape != src_k_scale.shape or
+                dst_k_scale.shape[0] != dst_k.shape[0] or src_k_scale.shape[0] != src_k.shape[0]):
+            raise ValueError("scale pools must be [num_blocks, ...] like their caches")
+        sbytes = _block_bytes(src_k_scale)
+        if _block_bytes(dst_k_scale) != sbytes:
+            raise ValueError("source and destination scale blocks differ in size")
     if pairs.dtype != torch.int32 or pairs.device.type != "cuda":
         raise TypeError("pairs must be an int32 CUDA tensor")
-    rc = N.lib().pkv_copy_blocks(
-        _any_ptr(dst_k), _any_ptr(dst_v), _any_ptr(src_k), _any_ptr(src_v), block_bytes,
-        dst_k.shape[0], src_k.shape[0], _any_ptr(dst_k_scale), _any_ptr(dst_v_scale),
-        _any_ptr(src_k_scale), _any_ptr(src_v_scale), sbytes, _ptr(pairs), pairs.shape[0],
-        _ptr(err_flag), _stream(stream))
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [num_pairs, 2]")
+    dev = pairs.get_device()
+    for t in (dst_k, dst_v, src_k, src_v, err_flag) + scales:
+        if t is not None and t.device.type == "cuda" and t.get_device() != dev:
+            raise ValueError("device pools, pairs and err_flag must be on one device")
+    rc = _on(dev, N.lib().pkv_copy_blocks,
+             _any_ptr(dst_k), _any_ptr(dst_v), _any_ptr(src_k), _any_ptr(src_v), block_bytes,
+             dst_k.shape[0], src_k.shape[0], _any_ptr(dst_k_scale), _any_ptr(dst_v_scale),
+             _any_ptr(src_k_scale), _any_ptr(src_v_scale), sbytes, _ptr(pairs), pairs.shape[0],
+             _ptr(err_flag), _stream(stream, dev))
     N.check(rc, "pkv_copy_blocks")
+
+
+def _block_bytes(pool: torch.Tensor) -> int:
+    return math.prod(pool.shape[1:]) * pool.element_size()
