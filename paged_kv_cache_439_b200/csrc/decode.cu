@@ -14,7 +14,7 @@
 // and `merge_kernel` combines the splits.
 //
 // Two engines:
-//  * mma (bf16 and int8 caches): per-warp cp.async stage rings; each stage is
+//  * mma (bf16, INT8 and FP8 caches): per-warp cp.async stage rings; each stage is
 //    read into registers as soon as it lands and refilled at once; scores and
 //    the PV update run on mma.sync m16n8k16 with fp32 accumulation.
 //  * simt (fp32 caches): per-warp cp.async rings, fp32 FMA dot products, two
@@ -184,12 +184,12 @@ __device__ __forceinline__ int phys_of(const DecodeParams& p, const CtaSetup& c,
   return t < c.t_end ? s_phys[(t >> p.log2_bs) - c.blk0] : -1;
 }
 
-// Issues the cp.async copies of one 16-token tile (K and V, plus INT8 scales)
+// Issues the cp.async copies of one 16-token tile of the fp32 engine (K and V)
 // into a stage of the calling warp's ring; one commit group per call.
-template <int HD, int ELEM, bool I8>
+template <int HD, int ELEM>
 __device__ __forceinline__ void load_tile(const DecodeParams& p, const CtaSetup& c,
                                           const int* s_phys, int tile_t0, uint8_t* k_st,
-                                          uint8_t* v_st, float* sc_st, int lane) {
+                                          uint8_t* v_st, int lane) {
   constexpr int ROWB = HD * ELEM;
   constexpr int CH = ROWB / 16;
   constexpr int PER_LANE = 16 * CH / kWarp;
@@ -214,19 +214,6 @@ __device__ __forceinline__ void load_tile(const DecodeParams& p, const CtaSetup&
     const uint32_t so = (uint32_t)swz<CH>(row, ch) * 16;
     cp_async_16(ks + so, kb + off, n);
     cp_async_16(vs + so, vb + off, n);
-  }
-  if constexpr (I8) {
-    const int row = lane & 15;
-    const int t = tile_t0 + row;
-    const int phys = phys_of(p, c, s_phys, t);
-    const float* src = (lane < 16) ? p.k_scale : p.v_scale;
-    size_t off = 0;
-    int n = 0;
-    if (phys >= 0) {
-      off = ((size_t)phys * p.num_kv_heads + c.kvh) * p.block_size + (t & (p.block_size - 1));
-      n = 4;
-    }
-    cp_async_4(smem_u32(sc_st + lane), src + off, n);
   }
   cp_async_commit();
 }
@@ -302,7 +289,7 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 
 
 // ---------------------------------------------------------------------------
-// mma engine: bf16 or int8 caches, q in bf16.
+// mma engine: bf16, INT8 or FP8 caches, q in bf16.
 //
 // Each warp streams its own interleaved 16-token tiles (the warp's tile i is
 // CTA tile warp + i * NWARPS) through a ring of NSTAGES cp.async stages.  As
@@ -920,9 +907,9 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
   for (int i = 0; i < NSTAGES - 1; ++i) {
     if (i < my_n)
-      load_tile<HD, ELEM, false>(p, c, s_phys, c.t_begin + (warp + i * NWARPS) * 16,
-                                 my_ring + (size_t)i * STAGE_B,
-                                 my_ring + (size_t)i * STAGE_B + TILE_B, nullptr, lane);
+      load_tile<HD, ELEM>(p, c, s_phys, c.t_begin + (warp + i * NWARPS) * 16,
+                          my_ring + (size_t)i * STAGE_B, my_ring + (size_t)i * STAGE_B + TILE_B,
+                          lane);
     else
       cp_async_commit();
   }
@@ -932,8 +919,8 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       const int ii = i + NSTAGES - 1;
       if (ii < my_n) {
         uint8_t* st = my_ring + (size_t)(ii % NSTAGES) * STAGE_B;
-        load_tile<HD, ELEM, false>(p, c, s_phys, c.t_begin + (warp + ii * NWARPS) * 16, st,
-                                   st + TILE_B, nullptr, lane);
+        load_tile<HD, ELEM>(p, c, s_phys, c.t_begin + (warp + ii * NWARPS) * 16, st,
+                            st + TILE_B, lane);
       } else {
         cp_async_commit();
       }
