@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--unfused", action="store_true",
                     help="time the step as two calls (kv_cache_append, then decode) instead of "
                          "the one-launch paged_attention_decode_append")
+    ap.add_argument("--append", action="store_true",
+                    help="time kv_cache_append: the workload's pre-fill tokens (up to 65,536) "
+                         "in one call, and the one-token-per-sequence decode append")
     ap.add_argument("--swap", action="store_true",
                     help="time swapping every sequence's blocks out to pinned host memory and "
                          "back (pkv_copy_blocks) against a plain pinned memcpy of the same bytes")
@@ -333,6 +336,69 @@ def device_cache(wl, dev):
     return tdt, k_cache, v_cache, k_scale, v_scale, err
 
 
+def _event_timer(stream):
+    """fn, reps -> mean ms per call on `stream` (three untimed calls first)."""
+    import torch
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+    return timed
+
+
+def run_append(args):
+    """Append bandwidth: the workload's pre-fill tokens (up to 65,536) written
+    by one kv_cache_append call, against the bytes it must move (K and V rows
+    read in the input dtype, written in the cache's, plus the scales of one-byte
+    caches); and the decode-step append of one token per sequence."""
+    import torch
+    import paged_kv_cache_439_b200 as pkv
+    from paged_kv_cache_439_b200.workloads import make_workload, workload_seed
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    extra = {"cache_dtype": args.kv_dtype} if args.kv_dtype else {}
+    wl = make_workload(args.workload, block_size=args.block_size,
+                       data_seed=workload_seed(args.workload), **extra)
+    _, k_cache, v_cache, ks, vs, err = device_cache(wl, dev)
+    T = min(wl.prefill_k.shape[0], 1 << 16)
+    bk, bv = wl.prefill_k[:T].to(dev), wl.prefill_v[:T].to(dev)
+    bsl = wl.prefill_slots[:T].to(dev)
+    nk, nv, ns = wl.new_k.to(dev), wl.new_v.to(dev), wl.new_slots.to(dev)
+    timed = _event_timer(torch.cuda.current_stream())
+    reps = max(1, min(args.steps, 50))
+    t_bulk = timed(lambda: pkv.kv_cache_append(bk, bv, bsl, k_cache, v_cache, ks, vs,
+                                               err_flag=err), reps)
+    t_step = timed(lambda: pkv.kv_cache_append(nk, nv, ns, k_cache, v_cache, ks, vs,
+                                               err_flag=err), 10 * reps)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"append kernel flagged {int(err.item())}")
+    per_tok = wl.num_kv_heads * wl.head_dim * 2 * (bk.element_size() + wl.cache_elem_bytes())
+    if ks is not None:
+        per_tok += wl.num_kv_heads * 2 * 4
+    peak, peak_src = measured_peak()
+    gbs = T * per_tok / (t_bulk * 1e-3) / 1e9
+    line = {"metric": "KV append GB/s (bytes read and written by one kv_cache_append call)",
+            "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": reps, "warmup": 3,
+            "higher_is_better": True,
+            "config": {"workload": wl.name, "cache_dtype": wl.cache_dtype, "tokens": T,
+                       "bytes_per_token": per_tok},
+            "frac_of_hbm_peak": round(gbs / peak, 3), "peak": peak, "peak_source": peak_src,
+            "bulk_ms": round(t_bulk, 4),
+            "decode_append_us": round(t_step * 1e3, 2), "decode_append_tokens": wl.num_seqs}
+    print(json.dumps(line), flush=True)
+
+
 def run_swap(args):
     """Swap bandwidth: every block of every sequence out to a pinned host pool
     in one pkv_copy_blocks launch, then back in, each timed with CUDA events;
@@ -362,20 +428,7 @@ def run_swap(args):
     nbytes = 2 * (hk.numel() * hk.element_size() + (hks.numel() * 4 if hks is not None else 0))
     flat_dev = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     flat_host = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
-    stream = torch.cuda.current_stream()
-
-    def timed(fn, reps):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / reps
-
+    timed = _event_timer(torch.cuda.current_stream())
     reps = max(1, min(args.steps, 20))
     t_out = timed(lambda: pkv.copy_blocks(hk, hv, k, v, out_pairs, hks, hvs, ks, vs,
                                           err_flag=err), reps)
@@ -405,6 +458,9 @@ def main():
         return
     if args.swap:
         run_swap(args)
+        return
+    if args.append:
+        run_append(args)
         return
     import torch
     import torch.distributed as dist
