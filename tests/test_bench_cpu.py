@@ -1,0 +1,72 @@
+"""The benchmark's CPU legs: the reference arm (the oracle timed on the host)
+and the CPU baseline, on the tiny workload.  They need no GPU, so the JSON
+contract of those lines is checked here."""
+import importlib.util
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench_module():
+    spec = importlib.util.spec_from_file_location("bench_under_test",
+                                                  os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _run(*args, env=None):
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                          capture_output=True, text=True, timeout=600, cwd=ROOT,
+                          env={**os.environ, **(env or {})})
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _run("--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "1")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 1
+    assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny" and "l2" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_is_silent_on_other_ranks():
+    r = _run("--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0",
+             env={"RANK": "1"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_cpu_baseline_reports_threads_and_one_thread():
+    bench = _bench_module()
+    cb = bench.run_cpu_baseline("tiny", None, 0.2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "GB/s" and cb["value"] > 0
+    assert cb["cores"] >= 1 and "tiny" in cb["sample"]
+    st = cb["single_thread"]
+    assert st["value"] > 0 and st["unit"] == "GB/s" and "one thread" in st["sample"]
+
+
+def test_l2_note_counts_shared_blocks_once():
+    bench = _bench_module()
+    from paged_kv_cache_439_b200.workloads import make_custom
+    shared = make_custom("l2-shared", [300, 300, 300], 4, 2, 64, 16, "bf16", seed=9,
+                         shared_prefix=256)
+    own = make_custom("l2-own", [300, 300, 300], 4, 2, 64, 16, "bf16", seed=9)
+    per_block = 16 * 2 * 64 * 2 * 2
+    n_shared = len(set(shared.block_tables[shared.block_tables >= 0].tolist()))
+    n_own = len(set(own.block_tables[own.block_tables >= 0].tolist()))
+    assert n_shared < n_own
+    assert f"distinct KV {n_shared * per_block // 10**6} MB" in bench.l2_note(shared)
+    assert "fits the 126 MB L2" in bench.l2_note(own)
