@@ -182,3 +182,51 @@ def test_workspace_sizes(lib):
     rows = 16 * 64 * s
     assert lib.pkv_workspace_size(16, 64, 8, 128, 32768, 1, 0) == \
         -(-rows * 128 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
+
+
+def _header_prototypes():
+    """name -> (return type, [parameter types]) for every declaration in pkv.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    protos = {}
+    for m in re.finditer(r"([A-Za-z_][\w \*]*?)\b(pkv_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        types = []
+        if params and params != "void":
+            for p in params.split(","):
+                p = " ".join(p.split())
+                # drop the parameter name: the last identifier not followed by '*'
+                types.append(re.sub(r"\s*\b\w+$", "", p) if not p.endswith("*") else p)
+        protos[name] = (ret, types)
+    return protos
+
+
+def _kind(c_type: str) -> str:
+    t = c_type.replace("const ", "").strip()
+    if "*" in t or t == "pkv_stream_t":
+        return "pointer"
+    return {"int": "int", "pkv_dtype": "int", "int32_t": "int", "int64_t": "int64",
+            "size_t": "size_t", "float": "float", "void": "void"}[t]
+
+
+def test_binding_prototypes_match_the_header():
+    """Each ctypes prototype has the header's parameter count and, position by
+    position, the same kind of type, so no argument is passed in the wrong
+    register or width."""
+    import ctypes
+    from paged_kv_cache_439_b200 import _native
+    kind_of = {ctypes.c_void_p: "pointer", ctypes.c_char_p: "pointer", ctypes.c_int: "int",
+               ctypes.c_int32: "int", ctypes.c_int64: "int64", ctypes.c_size_t: "size_t",
+               ctypes.c_float: "float", None: "void"}
+
+    def ck(t):
+        if t in kind_of:
+            return kind_of[t]
+        return "pointer" if issubclass(t, ctypes._Pointer) else repr(t)
+
+    protos = _header_prototypes()
+    assert set(protos) == set(_native.SIGNATURES)
+    for name, (res, args) in _native.SIGNATURES.items():
+        ret, params = protos[name]
+        assert [ck(a) for a in args] == [_kind(p) for p in params], name
+        assert ck(res) == _kind(ret), name
