@@ -230,3 +230,22 @@ def test_binding_prototypes_match_the_header():
         ret, params = protos[name]
         assert [ck(a) for a in args] == [_kind(p) for p in params], name
         assert ck(res) == _kind(ret), name
+
+
+@pytest.mark.parametrize("cache_dt", [0, 1, 2, 3])
+def test_split_plans_cover_the_context_in_bounded_chunks(lib, cache_dt):
+    """For every shape the automatic split count covers max_context_len with
+    16-token-aligned chunks of at most 8192 tokens (the block-table slice a CTA
+    stages in shared memory), and the workspace size matches that count."""
+    def ceil(a, b):
+        return -(-a // b)
+    for max_ctx in (1, 15, 16, 17, 255, 256, 4096, 8192, 8193, 32768, 100_000, 1 << 20):
+        for num_seqs in (1, 2, 16, 64, 512):
+            for nkv in (1, 8, 40):
+                s = lib.pkv_decode_num_splits(num_seqs, nkv, 128, max_ctx, cache_dt)
+                assert s >= max(1, ceil(max_ctx, 8192)), (max_ctx, num_seqs, nkv, s)
+                chunk = ceil(ceil(max_ctx, s), 16) * 16
+                assert chunk <= 8192 and s * chunk >= max_ctx and (s - 1) * chunk < max_ctx
+                rows = num_seqs * nkv * s
+                want = 0 if s == 1 else ceil(rows * 128 * 4, 256) * 256 + ceil(rows * 4, 256) * 256
+                assert lib.pkv_workspace_size(num_seqs, nkv, nkv, 128, max_ctx, cache_dt, 0) == want
