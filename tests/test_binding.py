@@ -229,3 +229,16 @@ def test_binding_passes_shared_prefix_sizes(fake):
     name, a = fake.calls[-1]
     assert name == "pkv_paged_attention_decode_shared_prefix_append"
     assert a[13:17] == (B, nq, nkv, d) and a[20] == 128
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without libpkv.so every call raises: there is no fallback path."""
+    from paged_kv_cache_439_b200 import _native
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "libpkv.so"))
+    with pytest.raises(ImportError, match="libpkv.so not found"):
+        pkv.decode_num_splits(4, 8, 128, 4096, torch.bfloat16)
+    with pytest.raises(ImportError, match="libpkv.so not found"):
+        pkv.workspace_size(4, 32, 8, 128, 4096, torch.bfloat16)
+    with pytest.raises(ImportError, match="libpkv.so not found"):
+        pkv.BlockManager(16, 16)
