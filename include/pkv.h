@@ -288,8 +288,14 @@ int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream);
  *   - Every call shares the array: calls whose kernels overlap on the GPU
  *     (e.g. on different streams) race and must be serialised by the caller.
  *     Nothing in the array has to start at zero.
- *   - The first call on each device looks up the array's device address with
- *     that device current; make that first call before any stream capture.
+ *   - The first call in each CUDA context (normally once per device) looks
+ *     up the array's device address with that device current and caches it
+ *     with the context's unique id; a call in a new context (for example after
+ *     cudaDeviceReset) looks it up again rather than reuse a stale address.
+ *   - The driver reserves the array's 16 MiB when it loads the module that
+ *     holds it; with lazy module loading (the CUDA default) that is this
+ *     first call, which can then fail with PKV_ERR_CUDA if the device has no
+ *     16 MiB left.  Make the first call at start-up, before any stream capture.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 int pkv_paged_attention_decode_noalloc(void* out, const void* q, pkv_dtype q_dt,

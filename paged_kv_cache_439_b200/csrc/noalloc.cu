@@ -19,10 +19,19 @@
 //  * The array keeps whatever the previous call left.  Nothing has to start at
 //    zero: every scratch entry the merge kernel reads is first written by the
 //    decode kernel of the same call.
-//  * The first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress, with that device current) and caches it; make that
-//    first call before any stream capture.
+//  * The first call in each CUDA context (normally once per device, the
+//    device's primary context) looks up the array's device address
+//    (cudaGetSymbolAddress, with that device current) and caches it together
+//    with the context's unique id.  A later call in another context (after a
+//    cudaDeviceReset, for example, which makes the module load again and can
+//    move the array) looks the address up afresh instead of reusing it.
+//  * The driver reserves the array's 16 MiB when it loads the module that
+//    holds it.  With lazy module loading (the CUDA default) that happens at
+//    this first call, which can therefore fail with PKV_ERR_CUDA when the
+//    device has no 16 MiB left.  Make the first call at start-up, before any
+//    stream capture.
 //  * Nothing here calls cudaMalloc, cudaFree or an allocating library routine.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -35,21 +44,53 @@ static __device__ __align__(256) unsigned char g_decode_scratch[PKV_NOALLOC_SCRA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices];  // device address of g_decode_scratch, per device
+struct ScratchSlot {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to
+  void* addr;                 // device address of g_decode_scratch in that context
+};
+ScratchSlot g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the current device (set-up on first use).
+// cuCtxGetId (unique per context for the life of the process, never reused)
+// through the runtime's driver entry point, so the library does not link
+// against libcuda.  Null when the driver does not provide it.
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetIdFn ctx_get_id() {
+  static CtxGetIdFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetIdFn>(ptr);
+  });
+  return fn;
+}
+
+// Device address of the scratch array in the current context.  The lookup is
+// made once per context and cached per device with the context's id; when the
+// id cannot be read the address is looked up on every call.
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_UNSUPPORTED;
+  // (no context current yet: the id read fails and the address is looked up,
+  // which also makes the device's primary context current)
+  unsigned long long id = 0;
+  const CtxGetIdFn get_id = ctx_get_id();
+  const bool have_id = get_id != nullptr && get_id(nullptr, &id) == CUDA_SUCCESS && id != 0;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) return PKV_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+  if (have_id && g_scratch[dev].addr != nullptr && g_scratch[dev].ctx_id == id) {
+    *out = g_scratch[dev].addr;
+    return PKV_OK;
   }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) return PKV_ERR_CUDA;
+  g_scratch[dev].ctx_id = have_id ? id : 0;
+  g_scratch[dev].addr = have_id ? p : nullptr;
+  *out = p;
   return PKV_OK;
 }
 

@@ -246,6 +246,19 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Bounded wait for the phase that tile `last` completed on a two-stage ring's
+// barrier pair (tile j: stage j % 2, phase j / 2), and, when both stages were
+// used, for the other stage's last tile.  True when nothing was issued.
+__device__ __forceinline__ bool drain_last(uint32_t bar_pair, int last) {
+  bool done = true;
+  for (int j = last; j >= 0 && j >= last - 1; --j)
+    done = done && mbar_wait(bar_pair + 8 * (j % 2), (uint32_t)((j / 2) & 1));
+  return done;
+}
+
+// Bits of the CTA's failure word: a wait gave up; a drain gave up as well.
+constexpr int kFailWait = 1, kFailDrain = 2;
+
 template <int HD>
 __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs per SM partition
     prefix_kernel(const DecodeParams p, const PrefixParams pp,
@@ -367,6 +380,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       };
       auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
       auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
+      int k_last = -1, v_last = -1;  // last K and V tile issued
       // Q with K0 first (S of tile 0 waits for them), then V0, K1, V1
       mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
 #pragma unroll
@@ -374,23 +388,37 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
         tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
       load_tile(&tm_k, kstage(0), 0, bar_k);
       load_tile(&tm_v, vstage(0), 0, bar_v);
+      k_last = v_last = 0;
       if (ntiles > 1) {
         load_tile(&tm_k, kstage(1), 1, bar_k + 8);
         load_tile(&tm_v, vstage(1), 1, bar_v + 8);
+        k_last = v_last = 1;
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         // S of tile j is done: K tile j's stage takes tile j + 2
         if (j + 2 < ntiles) {
           ok = mbar_wait(bar_kfree + 8 * (j % 2), (uint32_t)((j / 2) & 1));
-          if (ok) load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
+          if (ok) {
+            load_tile(&tm_k, kstage(j), j + 2, bar_k + 8 * (j % 2));
+            k_last = j + 2;
+          }
         }
         // P V of tile j - 1 is done: its V stage takes tile j + 1
         if (ok && j > 0 && j + 1 < ntiles) {
           ok = mbar_wait(bar_vfree + 8 * ((j - 1) % 2), (uint32_t)(((j - 1) / 2) & 1));
-          if (ok) load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
+          if (ok) {
+            load_tile(&tm_v, vstage(j + 1), j + 1, bar_v + 8 * ((j + 1) % 2));
+            v_last = j + 1;
+          }
         }
       }
-      if (!ok) *s_fail = 1;
+      if (!ok) atomicOr(const_cast<int*>(s_fail), kFailWait);
+      // Drain: every copy this lane issued lands before the CTA can exit, also
+      // after a wait gave up.  Tile j of a ring completes phase j / 2 of its
+      // stage's barrier, and only this lane's loads arrive there, so waiting
+      // on the parity of the last tile issued per stage cannot alias.
+      if (!drain_last(bar_k, k_last) || !drain_last(bar_v, v_last))
+        atomicOr(const_cast<int*>(s_fail), kFailDrain);
     }
   } else if (mma_warp) {
     // ================= MMA warp: one lane issues every tcgen05.mma ============
@@ -424,24 +452,43 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
         mma_commit(bar_odone);
         mma_commit(bar_vfree + 8 * (j % 2));
       };
+      int n_qk = 0, n_pv = 0;  // tiles whose S = Q K^T / O += P V were issued
       ok = mbar_wait(bar_k, 0);
       tc_fence_after();
-      if (ok) issue_qk(0);
+      if (ok) {
+        issue_qk(0);
+        n_qk = 1;
+      }
       for (int j = 0; ok && j < ntiles; ++j) {
         // every row has read S_j: S of tile j + 1 may overwrite it
         ok = mbar_wait(bar_sfree, (uint32_t)(j & 1));
         tc_fence_after();
         if (ok && j + 1 < ntiles) {
           ok = mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
-          if (ok) issue_qk(j + 1);
+          if (ok) {
+            issue_qk(j + 1);
+            n_qk = j + 2;
+          }
         }
         // every row has written P_j, V_j has landed: O += P_j V_j
         if (ok) ok = mbar_wait(bar_pfull, (uint32_t)(j & 1));
         if (ok) ok = mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
         tc_fence_after();
-        if (ok) issue_pv(j);
+        if (ok) {
+          issue_pv(j);
+          n_pv = j + 1;
+        }
       }
-      if (!ok) *s_fail = 1;
+      if (!ok) atomicOr(const_cast<int*>(s_fail), kFailWait);
+      // Drain, also after a wait gave up: the last phase committed on each
+      // barrier completes only once every MMA issued before that commit has
+      // finished and its arrive has landed.  Only this lane commits to these
+      // barriers, so none of them can be past the phase waited for.
+      bool drained = true;
+      if (n_qk > 0) drained = drained && mbar_wait(bar_sfull, (uint32_t)((n_qk - 1) & 1));
+      if (n_pv > 0) drained = drained && mbar_wait(bar_odone, (uint32_t)((n_pv - 1) & 1));
+      drained = drained && drain_last(bar_kfree, n_qk - 1) && drain_last(bar_vfree, n_pv - 1);
+      if (!drained) atomicOr(const_cast<int*>(s_fail), kFailDrain);
     }
   } else {
     // ================= softmax: thread r owns row r ==========================
@@ -553,7 +600,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     // ---- the last P V
     ok = ok && warp_wait(bar_odone, (uint32_t)((ntiles - 1) & 1));
     tc_fence_after();
-    if (!ok) *s_fail = 1;
+    if (!ok && lane == 0) atomicOr(const_cast<int*>(s_fail), kFailWait);
     // ---- normalise this slice's partial into shared memory (the K/V rings,
     // idle once the last P V is done), so that whole rows go out coalesced
     if (ok) {
@@ -578,8 +625,10 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
   }
 
   tc_fence_before();
-  const bool failed = __syncthreads_or(!ok || *s_fail);
-  if (!failed && warp < kTcSoftmaxWarps) {  // coalesced rows of the workspace
+  const bool failed = __syncthreads_or(!ok || *s_fail != 0);
+  if (warp < kTcSoftmaxWarps) {  // coalesced rows of the workspace
+    // A slice that gave up writes a defined partial instead (o = 0, log2-sum-exp
+    // = -inf): the merge then gives it weight 0 and the output stays finite.
     constexpr int CHK = HD / 4;
     constexpr int RPI = 32 / CHK;  // rows per warp store
     const float4* stage = reinterpret_cast<const float4*>(gbase + Cfg::Q_BYTES);
@@ -588,10 +637,15 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       if (rr >= spc * G || sq >= p.num_seqs) continue;
       const size_t slot = ((size_t)sq * p.num_q_heads + kvh * G + rr % G) * p.ws_slots + split;
       const int ch = lane % CHK;
-      reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] = stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
+      reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] =
+          failed ? make_float4(0.f, 0.f, 0.f, 0.f) : stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
+      if (failed && ch == 0) p.ws_lse[slot] = -CUDART_INF_F;
     }
   }
   if (failed && tid == 0) set_flag(p.err_flag, PKV_FLAG_TIMEOUT);
+  // Tensor memory is freed after the bounded drains above, also when one of
+  // them gave up: tcgen05.alloc waits without a bound for free columns, so
+  // memory left allocated could stall a later CTA on this SM indefinitely.
   if (warp == 0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),

@@ -466,3 +466,80 @@ def test_copy_blocks_definition():
     assert (dst[1] == -1).all() and (dst[2] == -1).all()
     with pytest.raises(oracle.OracleError):
         oracle.copy_blocks(dst, src, np.array([[5, 0]], dtype=np.int32))
+
+
+def _torch_e4m3_codes(y32: np.ndarray) -> np.ndarray:
+    """torch's float8_e4m3fn rounding (a library codec) of fp32 values, as bytes."""
+    return torch.from_numpy(np.ascontiguousarray(y32, dtype=np.float32)).to(
+        torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _fp32_tie_rows(rng, n_rows=24, d=128):
+    """Rows whose fp32 product x*scale lands exactly on a midpoint between two
+    E4M3 values while the exact (fp64) product does not: encoding the fp64
+    product, or rounding it twice, gives another code on these elements."""
+    mids = []
+    vals = sorted({oracle.e4m3_decode(c) for c in range(0x7F)
+                   if not math.isnan(oracle.e4m3_decode(c))})
+    for a, b in zip(vals[1:-1], vals[2:]):
+        mids.append((a + b) / 2)
+    rows, found = [], 0
+    while len(rows) < n_rows:
+        absmax = np.float32(rng.uniform(0.5, 20.0))
+        s = np.float32(np.float32(448.0) / absmax)
+        x = rng.standard_normal(d).astype(np.float32) * (absmax / 4)
+        x[0] = absmax
+        x = np.clip(x, -absmax, absmax)
+        hits = 0
+        for i in range(1, d):
+            m = float(rng.choice(mids)) * (1 if rng.random() < 0.5 else -1)
+            c0 = np.float32(m / float(s))
+            for c in (c0, np.nextafter(c0, np.float32(np.inf)), np.nextafter(c0, np.float32(-np.inf))):
+                p32 = np.float32(c) * s
+                if abs(float(c)) <= float(absmax) and float(p32) == m and float(c) * float(s) != m:
+                    x[i] = c
+                    hits += 1
+                    break
+        if hits:
+            found += hits
+            rows.append(x)
+    return np.stack(rows), found
+
+
+def test_quantize_fp8_codes_equal_library_rounding_of_fp32_products():
+    """FP8 rule (reading of the serving pages' --kv-cache-dtype fp8 flag, with the
+    mlqm page's §4 per-token scale rule carried over): codes are the E4M3
+    rounding, to nearest even with saturation, of the fp32 products x*scale.
+    The oracle's codes must equal torch's float8_e4m3fn conversion of exactly
+    those products, bit for bit (sign of zero included)."""
+    rng = np.random.default_rng(439)
+    rows = [rng.standard_normal(128).astype(np.float32) for _ in range(200)]
+    for _ in range(100):                       # 1% outliers x8, as in the 13B workload
+        x = rng.standard_normal(128).astype(np.float32)
+        x[rng.random(128) < 0.01] *= 8
+        rows.append(x)
+    for _ in range(50):                        # products in the subnormal range and -0
+        x = (rng.standard_normal(128) * 1e-4).astype(np.float32)
+        x[0] = np.float32(3.0)
+        x[1] = np.float32(-1e-9)
+        rows.append(x)
+    ties, n_ties = _fp32_tie_rows(rng)
+    assert n_ties >= 100                       # the constructed cases are really there
+    rows.extend(list(ties))
+    for x in rows:
+        codes, s = oracle.quantize_row_fp8(x)
+        assert s == np.float32(np.float32(448.0) / np.float32(np.abs(x).max()))
+        prod32 = x * s                          # numpy fp32 multiply: correctly rounded
+        assert np.array_equal(codes, _torch_e4m3_codes(prod32))
+    # the tie rows separate the fp32 reading from the fp64 one: on some of their
+    # elements the E4M3 value nearest the exact product is not the one chosen
+    vals = np.array(sorted({oracle.e4m3_decode(c) for c in range(0x7F)
+                            if not math.isnan(oracle.e4m3_decode(c))}))
+    differ = 0
+    for x in ties:
+        codes, s = oracle.quantize_row_fp8(x)
+        prod64 = x.astype(np.float64) * np.float64(s)
+        for p, c in zip(prod64, codes):
+            nearest = vals[np.argmin(np.abs(vals - abs(p)))]
+            differ += nearest != abs(oracle.e4m3_decode(int(c)))
+    assert differ >= 20
