@@ -27,7 +27,7 @@
  *                    pkv_shared_prefix_workspace_size
  *   block manager    pkv_bm_* (host bookkeeping: blocks, ref counts, fork,
  *                    copy-on-write, swap), pkv_copy_blocks (block copies)
- *   misc             pkv_copy, pkv_strerror, pkv_version
+ *   misc             pkv_copy, pkv_read, pkv_strerror, pkv_version
  *
  * Conventions shared by every call:
  *   - The caller allocates and owns every device buffer; the GPU calls keep no
@@ -268,6 +268,18 @@ int pkv_paged_attention_decode_shared_prefix_append(
  * process as the attention kernels.  Not part of the attention path.
  */
 int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream);
+
+/*
+ * pkv_read - streaming read of `bytes` bytes (a multiple of 16) at `src`
+ * (device, 16-byte aligned), folded by XOR into the device word *sink (4-byte
+ * aligned; the call XORs into it, so its value only keeps the loads alive).
+ * Used to measure the attainable HBM read bandwidth in the same process as the
+ * attention kernels, and, over a buffer larger than the L2, to flush the L2
+ * between timed calls: its loads allocate in L2 and write nothing, so no dirty
+ * line is left for the next call to write back.  Not part of the attention
+ * path.  Returns PKV_ERR_ARG for a null pointer or a size not a multiple of 16.
+ */
+int pkv_read(const void* src, size_t bytes, unsigned int* sink, pkv_stream_t stream);
 
 /* Bytes of the fixed device scratch behind pkv_paged_attention_decode_noalloc. */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)

@@ -47,6 +47,7 @@ SIGNATURES = {
                                                       _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                                       _i, _vp, _sz, _i, _vp, _vp]),
     "pkv_copy": (_i, [_vp, _vp, _sz, _vp]),
+    "pkv_read": (_i, [_vp, _sz, _vp, _vp]),
     "pkv_copy_blocks": (_i, [_vp, _vp, _vp, _vp, _sz, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp, _i,
                              _vp, _vp]),
     "pkv_bm_create": (_i, [_i, _i, ctypes.POINTER(ctypes.c_void_p)]),

@@ -375,6 +375,20 @@ def paged_attention_decode_shared_prefix_append(
     return out
 
 
+def read(src: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
+    """Streaming read of all of `src` (HBM read-bandwidth probe; over a buffer
+    larger than the L2 it also flushes the L2), XOR-folded into the int32
+    device word `sink`."""
+    if sink.dtype != torch.int32 or sink.numel() < 1:
+        raise ValueError("sink must hold one int32")
+    dev = _device(src)
+    if _device(sink) != dev:
+        raise ValueError("src and sink must be on one device")
+    rc = _on(dev, N.lib().pkv_read, _ptr(src, dev), _nbytes(src), _ptr(sink, dev),
+             _stream(stream, dev))
+    N.check(rc, "pkv_read")
+
+
 def copy(dst: torch.Tensor, src: torch.Tensor, stream=None) -> None:
     """Streaming device copy (HBM bandwidth probe)."""
     nbytes = _nbytes(src)

@@ -512,6 +512,13 @@ int pkv_paged_attention_decode_shared_prefix_append(
                             num_splits, err_flag, stream, k, v, slot_mapping);
 }
 
+int pkv_read(const void* src, size_t bytes, unsigned int* sink, pkv_stream_t stream) {
+  if (!src || !sink) return PKV_ERR_ARG;
+  if (bytes % 16) return PKV_ERR_ARG;
+  if (!aligned(src, 16) || !aligned(sink, 4)) return PKV_ERR_ALIGN;
+  return map_cuda(pkv::launch_read(src, bytes, sink, sm_count(), (cudaStream_t)stream));
+}
+
 int pkv_copy(void* dst, const void* src, size_t bytes, pkv_stream_t stream) {
   if (!dst || !src) return PKV_ERR_ARG;
   if (bytes % 16) return PKV_ERR_ARG;

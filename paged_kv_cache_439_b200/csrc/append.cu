@@ -251,6 +251,47 @@ __global__ void __launch_bounds__(256) copy_kernel(uint4* __restrict__ dst,
   for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
 }
 
+// Streaming read (HBM read-bandwidth probe, and an L2 flush that leaves only
+// clean lines behind): grid-stride 16-byte loads that allocate in L2, eight in
+// flight per thread, folded by XOR into one word per CTA so that no load is
+// dead.
+__global__ void __launch_bounds__(256) read_kernel(const uint4* __restrict__ src, size_t n,
+                                                   unsigned int* __restrict__ sink) {
+  constexpr int kIn = 8;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  unsigned int x = 0;
+  for (; i + (kIn - 1) * stride < n; i += kIn * stride) {
+    uint4 v[kIn];
+#pragma unroll
+    for (int j = 0; j < kIn; ++j) v[j] = __ldcg(src + i + j * stride);
+#pragma unroll
+    for (int j = 0; j < kIn; ++j) x ^= v[j].x ^ v[j].y ^ v[j].z ^ v[j].w;
+  }
+  for (; i < n; i += stride) {
+    const uint4 v = __ldcg(src + i);
+    x ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x ^= __shfl_xor_sync(0xffffffffu, x, off);
+  __shared__ unsigned int s_x[8];
+  if (threadIdx.x % kWarp == 0) s_x[threadIdx.x / kWarp] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned int r = 0;
+    for (int w = 0; w < (int)(blockDim.x / kWarp); ++w) r ^= s_x[w];
+    atomicXor(sink, r);
+  }
+}
+
+cudaError_t launch_read(const void* src, size_t bytes, unsigned int* sink, int num_sms,
+                        cudaStream_t st) {
+  const size_t n = bytes / 16;
+  if (n == 0) return cudaSuccess;
+  read_kernel<<<num_sms * 8, 256, 0, st>>>(static_cast<const uint4*>(src), n, sink);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t st) {
   const size_t n = bytes / 16;
   if (n == 0) return cudaSuccess;

@@ -69,5 +69,7 @@ cudaError_t launch_append(const void* k, const void* v, const int64_t* slot_mapp
                           cudaStream_t st);
 
 cudaError_t launch_copy(void* dst, const void* src, size_t bytes, int num_sms, cudaStream_t st);
+cudaError_t launch_read(const void* src, size_t bytes, unsigned int* sink, int num_sms,
+                        cudaStream_t st);
 
 }  // namespace pkv

@@ -68,5 +68,35 @@ def test_l2_note_counts_shared_blocks_once():
     n_shared = len(set(shared.block_tables[shared.block_tables >= 0].tolist()))
     n_own = len(set(own.block_tables[own.block_tables >= 0].tolist()))
     assert n_shared < n_own
-    assert f"distinct KV {n_shared * per_block // 10**6} MB" in bench.l2_note(shared)
-    assert "fits the 126 MB L2" in bench.l2_note(own)
+    assert f"distinct KV {n_shared * per_block // 10**6} MB" in bench.l2_note(shared, False)
+    assert "fits the 126 MB L2" in bench.l2_note(own, False)
+    assert "not flushed" in bench.l2_note(own, False)
+    assert "flushed between steps" in bench.l2_note(own, True)
+    assert bench.unique_kv_bytes(shared) == n_shared * per_block
+
+
+def test_bench_oracle_arm_matches_the_test_oracle_cache():
+    """The bench's CPU legs build the oracle's cache themselves (they do not
+    import the test helpers); on the same workload they give the same output."""
+    import numpy as np
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from pkv_testlib import OracleCache
+    from paged_kv_cache_439_b200.workloads import make_custom, make_workload
+    bench = _bench_module()
+    for wl in (make_workload("tiny"),
+               make_custom("arm-i8", [40, 300], 8, 2, 64, 16, "i8", seed=3, outlier_prob=0.01),
+               make_custom("arm-bf16", [17, 100], 8, 4, 128, 16, "bf16", seed=4)):
+        a = bench.OracleArm(wl).fill().decode()
+        b = OracleCache(wl).fill().decode()
+        assert np.array_equal(a, b)
+
+
+def test_reference_config_equals_the_gpu_arm_config_keys():
+    """Both arms describe the workload with the same config (no planner output in it)."""
+    bench = _bench_module()
+    from paged_kv_cache_439_b200.workloads import make_workload
+    args = bench.parse(["--workload", "tiny"])
+    c = bench.config_dict(make_workload("tiny"), args)
+    assert "num_splits" not in c and c["workload"] == "tiny"
+    assert c == bench.config_dict(make_workload("tiny"), args, flushed=True)
+    assert bench.parse([]).workload == "llama2-70b-gqa"

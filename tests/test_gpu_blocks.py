@@ -126,3 +126,23 @@ def test_bad_pairs_flag_and_skip():
     torch.cuda.synchronize()
     assert g.flags() & pkv.PKV_FLAG_BAD_BLOCK
     assert np.array_equal(bits(g.k), before)
+
+
+def test_probe_kernels_copy_and_read():
+    """The two in-process HBM probes: pkv_copy moves every byte (ragged size,
+    not a multiple of the grid), pkv_read XOR-folds every 16-byte vector."""
+    import paged_kv_cache_439_b200 as pkv
+    n = (3 << 20) + 16 * 37
+    src = torch.randint(-2**31, 2**31 - 1, (n // 4,), dtype=torch.int32, device="cuda")
+    dst = torch.zeros_like(src)
+    pkv.copy(dst, src)
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pkv.read(src, sink)
+    pkv.read(src, sink)      # XOR twice: back to zero
+    torch.cuda.synchronize()
+    assert torch.equal(dst, src)
+    assert int(sink.item()) == 0
+    pkv.read(src, sink)
+    words = src.cpu().numpy().view(np.uint32)
+    expect = int(np.bitwise_xor.reduce(words))
+    assert int(sink.cpu().numpy().view(np.uint32)[0]) == expect
