@@ -206,26 +206,35 @@ class ClockSampler:
         return False
 
 
-def decode_source_digest() -> str:
-    src = os.path.join(ROOT, "paged_kv_cache_439_b200", "csrc", "decode.cu")
-    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+def kernel_sources(cache_dtype):
+    """The source files the decode kernel of this cache format is built from."""
+    main = "decode_q8.cu" if cache_dtype in ("i8", "fp8") else "decode.cu"
+    return [main, "decode_common.cuh", "decode.cuh", "common.cuh"]
+
+
+def kernel_source_digest(cache_dtype) -> str:
+    h = hashlib.sha256()
+    for name in kernel_sources(cache_dtype):
+        with open(os.path.join(ROOT, "paged_kv_cache_439_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_record(wl):
     """DRAM bytes per decode launch of this workload from the committed ncu
-    records, or None when none matches it or decode.cu changed since the
-    capture."""
+    records, or None when none matches it or the kernel's sources changed
+    since the capture."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     try:
         with open(path) as f:
             recs = json.load(f).get("records", [])
     except Exception:
         return None
-    digest = decode_source_digest()
+    digest = kernel_source_digest(wl.cache_dtype)
     for rec in recs:
         if (rec.get("workload") == wl.name and rec.get("block_size") == wl.block_size and
                 rec.get("cache_dtype") == wl.cache_dtype and
-                rec.get("decode_cu_sha256_16") == digest):
+                rec.get("kernel_sources_sha256_16") == digest):
             return rec
     return None
 
@@ -491,15 +500,15 @@ def same_run_peaks(dev):
 
 def kernel_breakdown(call, flush, dev, reps=20):
     """Device time of each kernel of one call.  The call is captured into a
-    CUDA graph; each of its kernel nodes is re-launched from a graph of its
-    own, in the captured order, between CUDA events on one stream (L2 flushed
-    before each repetition).  Returns a list of {kernel, ms_mean, ms_median},
-    or {"error": ...} when the runtime bindings are not available."""
+    CUDA graph (driver API); each of its kernel nodes is re-launched from a
+    graph of its own, in the captured order, between CUDA events on one stream
+    (L2 flushed before each repetition).  Returns a list of {kernel, ms_mean,
+    ms_median}, or {"error": ...} when the bindings are not available."""
     import torch
     try:
-        from cuda.bindings import runtime as rt
+        from cuda.bindings import driver as cu
     except Exception as e:  # pragma: no cover - depends on the image
-        return {"error": f"cuda-python runtime bindings unavailable: {e}"}
+        return {"error": f"cuda-python driver bindings unavailable: {e}"}
 
     def ok(res, what):
         err = res[0] if isinstance(res, tuple) else res
@@ -507,54 +516,58 @@ def kernel_breakdown(call, flush, dev, reps=20):
             raise RuntimeError(f"{what}: {err}")
         return res[1:] if isinstance(res, tuple) and len(res) > 1 else None
 
-    graphs = []
+    graphs, execs = [], []
     try:
         s = torch.cuda.Stream(dev)
+        hs = cu.CUstream(s.cuda_stream)
         torch.cuda.synchronize()
         with torch.cuda.stream(s):
-            ok(rt.cudaStreamBeginCapture(
-                s.cuda_stream, rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed),
-               "begin capture")
+            ok(cu.cuStreamBeginCapture(
+                hs, cu.CUstreamCaptureMode.CU_STREAM_CAPTURE_MODE_RELAXED), "begin capture")
             try:
                 call()
             finally:
-                (graph,) = ok(rt.cudaStreamEndCapture(s.cuda_stream), "end capture")
+                (graph,) = ok(cu.cuStreamEndCapture(hs), "end capture")
         graphs.append(graph)
-        _, n = ok(rt.cudaGraphGetNodes(graph, 0), "node count")
-        nodes, _ = ok(rt.cudaGraphGetNodes(graph, n), "nodes")
-        # order the (linear) capture by its dependencies
-        order, seen = [], set()
-        deps = {}
+        _, n = ok(cu.cuGraphGetNodes(graph, 0), "node count")
+        nodes, _ = ok(cu.cuGraphGetNodes(graph, n), "nodes")
+        deps, byid = {}, {}
         for nd in nodes:
-            _, nd_n = ok(rt.cudaGraphNodeGetDependencies(nd, 0), "deps count")
-            d, _ = ok(rt.cudaGraphNodeGetDependencies(nd, nd_n), "deps") if nd_n else ([], 0)
+            byid[int(nd)] = nd
+            _, nd_n = ok(cu.cuGraphNodeGetDependencies(nd, 0), "deps count")
+            d = ok(cu.cuGraphNodeGetDependencies(nd, nd_n), "deps")[0] if nd_n else []
             deps[int(nd)] = [int(x) for x in d]
-        byid = {int(nd): nd for nd in nodes}
-        while len(order) < len(nodes):
+        order, seen = [], set()
+        while len(order) < len(nodes):  # the capture of one stream: a chain
             ready = [i for i in byid if i not in seen and all(x in seen for x in deps[i])]
             if not ready:
                 raise RuntimeError("capture is not a DAG")
             for i in ready:
                 seen.add(i)
                 order.append(byid[i])
-        execs, names = [], []
+        names = []
         for nd in order:
-            (typ,) = ok(rt.cudaGraphNodeGetType(nd), "node type")
-            if typ != rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+            (typ,) = ok(cu.cuGraphNodeGetType(nd), "node type")
+            if typ != cu.CUgraphNodeType.CU_GRAPH_NODE_TYPE_KERNEL:
                 continue
-            (params,) = ok(rt.cudaGraphKernelNodeGetParams(nd), "kernel params")
-            (g1,) = ok(rt.cudaGraphCreate(0), "graph create")
+            (params,) = ok(cu.cuGraphKernelNodeGetParams(nd), "kernel params")
+            (g1,) = ok(cu.cuGraphCreate(0), "graph create")
             graphs.append(g1)
-            ok(rt.cudaGraphAddKernelNode(g1, None, 0, params), "add kernel node")
-            (ex,) = ok(rt.cudaGraphInstantiate(g1, 0), "instantiate")
+            ok(cu.cuGraphAddKernelNode(g1, None, 0, params), "add kernel node")
+            (ex,) = ok(cu.cuGraphInstantiate(g1, 0), "instantiate")
             execs.append(ex)
             name = None
-            try:
-                res = rt.cudaFuncGetName(params.func)
-                if int(res[0]) == 0:
-                    name = res[1].decode() if isinstance(res[1], bytes) else str(res[1])
-            except Exception:
-                name = None
+            for getter, handle in ((getattr(cu, "cuFuncGetName", None), params.func),
+                                   (getattr(cu, "cuKernelGetName", None),
+                                    getattr(params, "kern", None))):
+                if name or getter is None or handle is None or int(handle) == 0:
+                    continue
+                try:
+                    res = getter(handle)
+                    if int(res[0]) == 0:
+                        name = res[1].decode() if isinstance(res[1], bytes) else str(res[1])
+                except Exception:
+                    name = None
             names.append(name or f"kernel {len(names)}")
         times = [[] for _ in execs]
         for _ in range(reps):
@@ -563,22 +576,25 @@ def kernel_breakdown(call, flush, dev, reps=20):
                 evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(execs) + 1)]
                 evs[0].record(s)
                 for i, ex in enumerate(execs):
-                    ok(rt.cudaGraphLaunch(ex, s.cuda_stream), "launch")
+                    ok(cu.cuGraphLaunch(ex, hs), "launch")
                     evs[i + 1].record(s)
             s.synchronize()
             for i in range(len(execs)):
                 times[i].append(evs[i].elapsed_time(evs[i + 1]))
-        for ex in execs:
-            rt.cudaGraphExecDestroy(ex)
         return [{"kernel": nm, "ms_mean": round(statistics.mean(t), 5),
                  "ms_median": round(statistics.median(t), 5)} for nm, t in zip(names, times)]
     except Exception as e:
         torch.cuda.synchronize()
         return {"error": repr(e)[:300]}
     finally:
+        for ex in execs:
+            try:
+                cu.cuGraphExecDestroy(ex)
+            except Exception:
+                pass
         for g in graphs:
             try:
-                rt.cudaGraphDestroy(g)
+                cu.cuGraphDestroy(g)
             except Exception:
                 pass
 

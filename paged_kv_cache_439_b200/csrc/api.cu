@@ -9,6 +9,10 @@
 
 namespace {
 
+#ifndef PKV_CASCADE_SUFFIX_FIRST
+#define PKV_CASCADE_SUFFIX_FIRST 1
+#endif
+
 constexpr int kMaxChunk = 8192;   // tokens per split (bounds the block-table slice in smem)
 constexpr int kMinChunk = 256;    // below this a split costs more than it balances
 constexpr int kTile = 16;         // tokens per tile of the decode kernels
@@ -470,8 +474,16 @@ int shared_prefix_impl(
   p.slot_mapping = slot_mapping;
 
   cudaStream_t st = (cudaStream_t)stream;
-  if (pkv::launch_prefix(p, pp, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
+#if PKV_CASCADE_SUFFIX_FIRST
+  // The suffix decode first; the prefix pass (independent of it: disjoint
+  // workspace slots, and the fused append never writes a shared block) is
+  // launched behind it and fills the SMs its last wave leaves idle.
   if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
+  if (pkv::launch_prefix(p, pp, head_dim, true, st) != cudaSuccess) return PKV_ERR_CUDA;
+#else
+  if (pkv::launch_prefix(p, pp, head_dim, false, st) != cudaSuccess) return PKV_ERR_CUDA;
+  if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
+#endif
   if (pkv::launch_merge(p, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }

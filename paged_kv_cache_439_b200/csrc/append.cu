@@ -13,7 +13,7 @@
 // code = clamp(rint(x * scale), -128, 127) in fp32 with round-half-to-even;
 // __fdiv_rn / __fmul_rn keep the division and the product correctly rounded
 // and unfused.  An all-zero row stores codes 0 and scale 1.  The FP8 variant
-// uses scale = 448 / max|x| and E4M3 codes (see append_fp8_kernel).
+// uses scale = 448 / max|x| and E4M3 codes (append_quant_kernel).
 #include "common.cuh"
 #include "decode.cuh"
 
@@ -56,144 +56,155 @@ __global__ void __launch_bounds__(kAppendThreads)
   }
 }
 
-template <typename T>
-__device__ __forceinline__ float to_f32(T x);
-template <>
-__device__ __forceinline__ float to_f32<float>(float x) {
-  return x;
-}
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
-  return __bfloat162float(x);
+// Quantising append (INT8 or FP8 cache).  One CTA of kQuantThreads threads
+// per token; a (tensor K|V, head) row of head_dim elements is held by a group
+// of kLanesPerRow lanes, lane j of the group holding elements EPL*j ..
+// EPL*j + EPL - 1 (EPL = head_dim / 8) with 16-byte vector loads, so one warp
+// works on four rows at once and the per-row steps (absmax reduction, the
+// scale division) are shared by those four.  The token's 2 * num_kv_heads
+// rows (K rows of every head, then V rows) are dealt to the groups; each lane
+// loads the rows of kQuantBatch passes before quantising any, so that many
+// row loads stay in flight.  The row rule is the one of quant_row_int8 /
+// quant_row_fp8 (common.cuh), written for the group layout: scale =
+// 127 / max|x| (448 / max|x| for FP8), correctly rounded; each code is the
+// correctly rounded fp32 product x * scale converted with round-to-nearest-
+// even and saturation (cvt.rni.sat.s8.f32, i.e. clamp(rint(.), -128, 127); for
+// FP8 cvt.rn.satfinite.e4m3x2); an all-zero row stores codes 0 and scale 1.
+constexpr int kQuantThreads = 256;
+constexpr int kLanesPerRow = 8;
+constexpr int kRowsPerPass = kQuantThreads / kLanesPerRow;  // 32 rows per CTA pass
+constexpr int kQuantBatch = 2;
+
+// One code of the INT8 rule from the fp32 product p: round half to even, then
+// saturate to [-128, 127].
+__device__ __forceinline__ uint32_t s8_code(float p) {
+  short q;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=h"(q) : "f"(p));
+  return (uint32_t)q & 0xFFu;
 }
 
-// One warp per (token, tensor K|V, head) row.  Lane l holds head_dim/32
-// consecutive elements.
-template <typename T, int HD>
-__global__ void __launch_bounds__(kAppendThreads)
-    append_int8_kernel(const T* __restrict__ k, const T* __restrict__ v,
-                       const int64_t* __restrict__ slot_mapping, int num_tokens,
-                       int num_kv_heads, int8_t* __restrict__ k_cache,
-                       int8_t* __restrict__ v_cache, float* __restrict__ k_scale,
-                       float* __restrict__ v_scale, int block_size, long long num_slots,
-                       int* err_flag) {
-  constexpr int E = HD / kWarp;  // elements per lane (2 or 4)
-  const int lane = threadIdx.x % kWarp;
-  const long long row = (long long)blockIdx.x * (kAppendThreads / kWarp) + threadIdx.x / kWarp;
-  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
-  if (row >= rows) return;
-  const int t = (int)(row / (2 * num_kv_heads));
-  const int rem = (int)(row % (2 * num_kv_heads));
-  const bool is_v = rem >= num_kv_heads;
-  const int h = is_v ? rem - num_kv_heads : rem;
+template <typename T, int EPL>
+__device__ __forceinline__ void widen_vecs(const uint4 (&v)[EPL * sizeof(T) / 16], float (&x)[EPL]) {
+  if constexpr (sizeof(T) == 2) {
+#pragma unroll
+    for (int i = 0; i < EPL / 8; ++i) {
+      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+        x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL / 4; ++i) {
+      x[4 * i] = __uint_as_float(v[i].x);
+      x[4 * i + 1] = __uint_as_float(v[i].y);
+      x[4 * i + 2] = __uint_as_float(v[i].z);
+      x[4 * i + 3] = __uint_as_float(v[i].w);
+    }
+  }
+}
+
+template <typename T, int HD, bool FP8>
+__global__ void __launch_bounds__(kQuantThreads)
+    append_quant_kernel(const T* __restrict__ k, const T* __restrict__ v,
+                        const int64_t* __restrict__ slot_mapping, int num_kv_heads,
+                        uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
+                        float* __restrict__ k_scale, float* __restrict__ v_scale, int log2_bs,
+                        long long num_slots, int* err_flag) {
+  constexpr int EPL = HD / kLanesPerRow;         // elements per lane: 16 or 8
+  constexpr int VECS = EPL * (int)sizeof(T) / 16;  // 16-byte loads per lane per row
+  constexpr int WORDS = EPL / 4;                 // 4-byte code words per lane per row
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
+  const int j = lane % kLanesPerRow;
   const long long slot = slot_mapping[t];
   if (slot < 0) return;
   if (slot >= num_slots) {
-    if (lane == 0 && h == 0 && !is_v) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
+    if (threadIdx.x == 0) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
     return;
   }
-  const T* src = (is_v ? v : k) + ((size_t)t * num_kv_heads + h) * HD + lane * E;
-  float x[E];
+  const int bs = 1 << log2_bs;
+  const long long blk = slot >> log2_bs;
+  const int off = (int)(slot & (bs - 1));
+  const int rows = 2 * num_kv_heads;
+  const size_t src_row0 = (size_t)t * num_kv_heads;
+  const size_t dst_row0 = (size_t)slot * num_kv_heads;
+  // every lane of a warp runs the same passes (the group shuffles need all 32)
+  for (int base = warp * (kWarp / kLanesPerRow); base < rows;
+       base += kRowsPerPass * kQuantBatch) {
+    uint4 buf[kQuantBatch][VECS];
 #pragma unroll
-  for (int e = 0; e < E; ++e) x[e] = to_f32(src[e]);
-  float scale;
-  const uint32_t packed = quant_row_int8<E>(x, &scale);
-  const long long blk = slot / block_size;
-  const int off = (int)(slot % block_size);
-  int8_t* dst = (is_v ? v_cache : k_cache) + ((size_t)slot * num_kv_heads + h) * HD + lane * E;
-  if constexpr (E == 4)
-    *reinterpret_cast<uint32_t*>(dst) = packed;
-  else
-    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
-  if (lane == 0) {
-    float* sc = is_v ? v_scale : k_scale;
-    sc[((size_t)blk * num_kv_heads + h) * block_size + off] = scale;
-  }
-}
-
-// FP8 (E4M3) variant of the same row rule: scale = 448 / max|x|, codes
-// E4M3(x * scale) with round-to-nearest-even and saturation (hardware cvt);
-// an all-zero row stores codes 0 and scale 1.
-template <typename T, int HD>
-__global__ void __launch_bounds__(kAppendThreads)
-    append_fp8_kernel(const T* __restrict__ k, const T* __restrict__ v,
-                      const int64_t* __restrict__ slot_mapping, int num_tokens, int num_kv_heads,
-                      uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
-                      float* __restrict__ k_scale, float* __restrict__ v_scale, int block_size,
-                      long long num_slots, int* err_flag) {
-  constexpr int E = HD / kWarp;  // elements per lane (2 or 4)
-  const int lane = threadIdx.x % kWarp;
-  const long long row = (long long)blockIdx.x * (kAppendThreads / kWarp) + threadIdx.x / kWarp;
-  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
-  if (row >= rows) return;
-  const int t = (int)(row / (2 * num_kv_heads));
-  const int rem = (int)(row % (2 * num_kv_heads));
-  const bool is_v = rem >= num_kv_heads;
-  const int h = is_v ? rem - num_kv_heads : rem;
-  const long long slot = slot_mapping[t];
-  if (slot < 0) return;
-  if (slot >= num_slots) {
-    if (lane == 0 && h == 0 && !is_v) set_flag(err_flag, PKV_FLAG_BAD_SLOT);
-    return;
-  }
-  const T* src = (is_v ? v : k) + ((size_t)t * num_kv_heads + h) * HD + lane * E;
-  float x[E];
+    for (int b = 0; b < kQuantBatch; ++b) {
+      const int r = base + lane / kLanesPerRow + b * kRowsPerPass;
+      if (r < rows) {
+        const bool is_v = r >= num_kv_heads;
+        const int h = is_v ? r - num_kv_heads : r;
+        const uint4* src =
+            reinterpret_cast<const uint4*>((is_v ? v : k) + (src_row0 + h) * HD) + j * VECS;
 #pragma unroll
-  for (int e = 0; e < E; ++e) x[e] = to_f32(src[e]);
-  float scale;
-  const uint32_t packed = quant_row_fp8<E>(x, &scale);
-  const long long blk = slot / block_size;
-  const int off = (int)(slot % block_size);
-  uint8_t* dst = (is_v ? v_cache : k_cache) + ((size_t)slot * num_kv_heads + h) * HD + lane * E;
-  if constexpr (E == 4)
-    *reinterpret_cast<uint32_t*>(dst) = packed;
-  else
-    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
-  if (lane == 0) {
-    float* sc = is_v ? v_scale : k_scale;
-    sc[((size_t)blk * num_kv_heads + h) * block_size + off] = scale;
+        for (int i = 0; i < VECS; ++i) buf[b][i] = __ldg(src + i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VECS; ++i) buf[b][i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < kQuantBatch; ++b) {
+      const int r = base + lane / kLanesPerRow + b * kRowsPerPass;
+      float x[EPL];
+      widen_vecs<T, EPL>(buf[b], x);
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(x[e]));
+#pragma unroll
+      for (int o = 1; o < kLanesPerRow; o <<= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float scale = amax > 0.f ? __fdiv_rn(FP8 ? 448.0f : 127.0f, amax) : 1.0f;
+      uint32_t w[WORDS];
+#pragma unroll
+      for (int q = 0; q < WORDS; ++q) {
+        const float p0 = __fmul_rn(x[4 * q], scale), p1 = __fmul_rn(x[4 * q + 1], scale);
+        const float p2 = __fmul_rn(x[4 * q + 2], scale), p3 = __fmul_rn(x[4 * q + 3], scale);
+        if constexpr (FP8)
+          w[q] = amax > 0.f ? (f32x2_to_e4m3x2(p0, p1) | (f32x2_to_e4m3x2(p2, p3) << 16)) : 0u;
+        else
+          w[q] = s8_code(p0) | (s8_code(p1) << 8) | (s8_code(p2) << 16) | (s8_code(p3) << 24);
+      }
+      if (r < rows) {
+        const bool is_v = r >= num_kv_heads;
+        const int h = is_v ? r - num_kv_heads : r;
+        uint8_t* dst = (is_v ? v_cache : k_cache) + (dst_row0 + h) * HD + j * EPL;
+        if constexpr (WORDS == 4)
+          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        else
+          *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+        if (j == 0) (is_v ? v_scale : k_scale)[((size_t)blk * num_kv_heads + h) * bs + off] = scale;
+      }
+    }
   }
 }
 
-template <typename T>
-cudaError_t launch_fp8(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
-                       int num_kv_heads, int head_dim, void* k_cache, void* v_cache,
-                       float* k_scale, float* v_scale, int block_size, long long num_slots,
-                       int* err_flag, cudaStream_t st) {
-  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
-  const long long per = kAppendThreads / kWarp;
-  const unsigned grid = (unsigned)((rows + per - 1) / per);
+template <typename T, bool FP8>
+cudaError_t launch_quant(const void* k, const void* v, const int64_t* slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim, void* k_cache,
+                         void* v_cache, float* k_scale, float* v_scale, int block_size,
+                         long long num_slots, int* err_flag, cudaStream_t st) {
+  int log2_bs = 0;
+  while ((1 << log2_bs) < block_size) ++log2_bs;
+  const dim3 grid((unsigned)num_tokens);
+  constexpr int threads = kQuantThreads;
   if (head_dim == 128)
-    append_fp8_kernel<T, 128><<<grid, kAppendThreads, 0, st>>>(
-        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
-        num_kv_heads, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale,
-        v_scale, block_size, num_slots, err_flag);
+    append_quant_kernel<T, 128, FP8><<<grid, threads, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_kv_heads,
+        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale, v_scale,
+        log2_bs, num_slots, err_flag);
   else
-    append_fp8_kernel<T, 64><<<grid, kAppendThreads, 0, st>>>(
-        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
-        num_kv_heads, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale,
-        v_scale, block_size, num_slots, err_flag);
-  return cudaGetLastError();
-}
-
-template <typename T>
-cudaError_t launch_i8(const void* k, const void* v, const int64_t* slot_mapping, int num_tokens,
-                      int num_kv_heads, int head_dim, void* k_cache, void* v_cache,
-                      float* k_scale, float* v_scale, int block_size, long long num_slots,
-                      int* err_flag, cudaStream_t st) {
-  const long long rows = (long long)num_tokens * 2 * num_kv_heads;
-  const long long per = kAppendThreads / kWarp;
-  const unsigned grid = (unsigned)((rows + per - 1) / per);
-  if (head_dim == 128)
-    append_int8_kernel<T, 128><<<grid, kAppendThreads, 0, st>>>(
-        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
-        num_kv_heads, static_cast<int8_t*>(k_cache), static_cast<int8_t*>(v_cache), k_scale,
-        v_scale, block_size, num_slots, err_flag);
-  else
-    append_int8_kernel<T, 64><<<grid, kAppendThreads, 0, st>>>(
-        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_tokens,
-        num_kv_heads, static_cast<int8_t*>(k_cache), static_cast<int8_t*>(v_cache), k_scale,
-        v_scale, block_size, num_slots, err_flag);
+    append_quant_kernel<T, 64, FP8><<<grid, threads, 0, st>>>(
+        static_cast<const T*>(k), static_cast<const T*>(v), slot_mapping, num_kv_heads,
+        static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache), k_scale, v_scale,
+        log2_bs, num_slots, err_flag);
   return cudaGetLastError();
 }
 
@@ -208,19 +219,21 @@ cudaError_t launch_append(const void* k, const void* v, const int64_t* slot_mapp
   const long long num_slots = (long long)num_blocks * block_size;
   if (cache_dt == PKV_FP8) {
     if (in_dt == PKV_BF16)
-      return launch_fp8<__nv_bfloat16>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
-                                       k_cache, v_cache, k_scale, v_scale, block_size,
-                                       num_slots, err_flag, st);
-    return launch_fp8<float>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim, k_cache,
-                             v_cache, k_scale, v_scale, block_size, num_slots, err_flag, st);
+      return launch_quant<__nv_bfloat16, true>(k, v, slot_mapping, num_tokens, num_kv_heads,
+                                               head_dim, k_cache, v_cache, k_scale, v_scale,
+                                               block_size, num_slots, err_flag, st);
+    return launch_quant<float, true>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                     k_cache, v_cache, k_scale, v_scale, block_size, num_slots,
+                                     err_flag, st);
   }
   if (cache_dt == PKV_I8) {
     if (in_dt == PKV_BF16)
-      return launch_i8<__nv_bfloat16>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
+      return launch_quant<__nv_bfloat16, false>(k, v, slot_mapping, num_tokens, num_kv_heads,
+                                                head_dim, k_cache, v_cache, k_scale, v_scale,
+                                                block_size, num_slots, err_flag, st);
+    return launch_quant<float, false>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim,
                                       k_cache, v_cache, k_scale, v_scale, block_size, num_slots,
                                       err_flag, st);
-    return launch_i8<float>(k, v, slot_mapping, num_tokens, num_kv_heads, head_dim, k_cache,
-                            v_cache, k_scale, v_scale, block_size, num_slots, err_flag, st);
   }
   const int elem = (in_dt == PKV_F32) ? 4 : 2;
   const int row_vecs = num_kv_heads * head_dim * elem / 16;

@@ -26,163 +26,9 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_common.cuh"
 
 namespace pkv {
-
-struct CtaSetup {
-  int seq, kvh, split;
-  int ctx;             // the sequence's (clamped) context length
-  int t_begin, t_end;  // token range of this CTA
-  int blk0;            // first logical block in s_phys
-  bool active;
-};
-
-// Clamped context length: identical in decode and merge kernels.
-__device__ __forceinline__ int effective_ctx(const DecodeParams& p, int seq, bool report) {
-  int ctx = p.context_lens[seq];
-  if (ctx < 0) {
-    if (report) set_flag(p.err_flag, PKV_FLAG_NEG_CTX);
-    ctx = 0;
-  }
-  const long long cap_tab = (long long)p.max_blocks_per_seq * p.block_size;
-  const long long cap_split = (long long)p.t_start + (long long)p.num_splits * p.chunk;
-  if (ctx > p.max_context_len || ctx > cap_tab) {
-    if (report) set_flag(p.err_flag, PKV_FLAG_CTX_RANGE);
-  }
-  long long c = ctx;
-  if (c > cap_tab) c = cap_tab;
-  if (c > cap_split) c = cap_split;
-  return (int)c;
-}
-
-// Loads and validates this CTA's slice of the block table into smem.
-__device__ __forceinline__ CtaSetup cta_setup(const DecodeParams& p, int* s_phys) {
-  CtaSetup c;
-  c.kvh = blockIdx.x;
-  c.seq = blockIdx.y;
-  c.split = blockIdx.z;
-  const bool report = (c.kvh == 0 && c.split == 0 && threadIdx.x == 0);
-  const int ctx = effective_ctx(p, c.seq, report);
-  c.t_begin = p.t_start + c.split * p.chunk;
-  c.ctx = ctx;
-  c.t_end = min(ctx, c.t_begin + p.chunk);
-  c.active = c.t_begin < c.t_end;
-  c.blk0 = c.t_begin >> p.log2_bs;
-  if (c.active) {
-    const int nphys = ((c.t_end - 1) >> p.log2_bs) - c.blk0 + 1;
-    const int32_t* row = p.block_tables + (size_t)c.seq * p.max_blocks_per_seq;
-    for (int i = threadIdx.x; i < nphys; i += blockDim.x) {
-      int b = row[c.blk0 + i];
-      if (b < 0 || b >= p.num_blocks) {
-        set_flag(p.err_flag, PKV_FLAG_BAD_BLOCK);
-        b = -1;
-      }
-      s_phys[i] = b;
-    }
-  }
-  __syncthreads();
-  return c;
-}
-
-// Cache formats of the mma engine.
-constexpr int kQuantNone = 0;  // bf16 values
-constexpr int kQuantI8 = 1;    // int8 codes, fp32 scale per token per head
-constexpr int kQuantFp8 = 2;   // E4M3 codes, fp32 scale per token per head
-
-// Fused append (pkv_paged_attention_decode_append), in two parts.
-//
-// Prefetch, in every warp before the CTA's first barrier: each lane loads its
-// share of the sequence's new K and V rows of this KV head (bf16 rows: lane l
-// holds 16-byte chunk l of K, then of V; one-byte caches: lane l holds
-// elements E*l .. E*l+E-1 of K in .x/.y and of V in .z/.w, E = head_dim / 32)
-// and the token's slot, so their latency overlaps the CTA set-up.
-template <int HD, int QM>
-__device__ __forceinline__ uint4 fused_prefetch(const DecodeParams& p, long long* slot) {
-  uint4 r = make_uint4(0u, 0u, 0u, 0u);
-  *slot = -1;
-  if (p.new_k == nullptr) return r;
-  const int lane = threadIdx.x % kWarp;
-  const size_t base = ((size_t)blockIdx.y * p.num_kv_heads + blockIdx.x) * HD;
-  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(p.new_k) + base;
-  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(p.new_v) + base;
-  *slot = p.slot_mapping[blockIdx.y];
-  if constexpr (QM == kQuantNone) {
-    constexpr int V = HD / 8;  // 16-byte chunks of a bf16 row
-    if (lane < 2 * V) r = reinterpret_cast<const uint4*>(lane < V ? k : v)[lane % V];
-  } else if constexpr (HD / kWarp == 4) {
-    const uint2 a = reinterpret_cast<const uint2*>(k)[lane];
-    const uint2 b = reinterpret_cast<const uint2*>(v)[lane];
-    r = make_uint4(a.x, a.y, b.x, b.y);
-  } else {
-    r.x = reinterpret_cast<const uint32_t*>(k)[lane];
-    r.z = reinterpret_cast<const uint32_t*>(v)[lane];
-  }
-  return r;
-}
-
-// Commit, after the set-up: the warp that will read the 16-token tile holding
-// position ctx - 1 (tile i of the CTA belongs to warp i % NWARPS) writes the
-// token's K and V rows into slot_mapping[seq], quantised for one-byte caches
-// with the append kernels' own row rule, then syncs the warp, so that its
-// later cp.async reads of that position see the rows.  No other CTA reads the
-// position.  The slot must be the one the block table gives position ctx - 1;
-// otherwise nothing is written and PKV_FLAG_BAD_SLOT is set.  A negative slot
-// writes nothing.
-template <int HD, int QM, int NWARPS>
-__device__ __forceinline__ void fused_commit(const DecodeParams& p, const CtaSetup& c,
-                                             const int* s_phys, uint4 r, long long slot) {
-  if (p.new_k == nullptr || !c.active || c.t_end != c.ctx) return;
-  const int pos = c.ctx - 1;
-  const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
-  if (warp != ((pos - c.t_begin) >> 4) % NWARPS || slot < 0) return;
-  const int bs = p.block_size;
-  const int b = s_phys[(pos >> p.log2_bs) - c.blk0];
-  if (b < 0 || slot != (long long)b * bs + (pos & (bs - 1))) {
-    if (lane == 0) set_flag(p.err_flag, PKV_FLAG_BAD_SLOT);
-    return;
-  }
-  const size_t row = (size_t)slot * p.num_kv_heads + c.kvh;  // in head_dim units
-  if constexpr (QM == kQuantNone) {
-    constexpr int V = HD / 8;
-    if (lane < 2 * V) {
-      void* cache = const_cast<void*>(lane < V ? p.k_cache : p.v_cache);
-      reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(cache) + row * HD)[lane % V] = r;
-    }
-  } else {
-    constexpr int E = HD / kWarp;  // elements per lane
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {  // K, then V
-      const uint32_t w0 = t ? r.z : r.x, w1 = t ? r.w : r.y;
-      float x[E];
-      x[0] = __uint_as_float(w0 << 16);
-      x[1] = __uint_as_float(w0 & 0xFFFF0000u);
-      if constexpr (E == 4) {
-        x[2] = __uint_as_float(w1 << 16);
-        x[3] = __uint_as_float(w1 & 0xFFFF0000u);
-      }
-      float scale;
-      const uint32_t packed =
-          QM == kQuantI8 ? quant_row_int8<E>(x, &scale) : quant_row_fp8<E>(x, &scale);
-      uint8_t* dst = static_cast<uint8_t*>(const_cast<void*>(t ? p.v_cache : p.k_cache)) +
-                     row * HD + lane * E;
-      if constexpr (E == 4)
-        *reinterpret_cast<uint32_t*>(dst) = packed;
-      else
-        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
-      if (lane == 0) {
-        float* sc = const_cast<float*>(t ? p.v_scale : p.k_scale);
-        sc[((size_t)b * p.num_kv_heads + c.kvh) * bs + (pos & (bs - 1))] = scale;
-      }
-    }
-  }
-  __syncwarp();
-}
-
-// Physical block of token t (-1 when masked: past the range or bad block).
-__device__ __forceinline__ int phys_of(const DecodeParams& p, const CtaSetup& c,
-                                       const int* s_phys, int t) {
-  return t < c.t_end ? s_phys[(t >> p.log2_bs) - c.blk0] : -1;
-}
 
 // Issues the cp.async copies of one 16-token tile of the fp32 engine (K and V)
 // into a stage of the calling warp's ring; one commit group per call.
@@ -218,74 +64,6 @@ __device__ __forceinline__ void load_tile(const DecodeParams& p, const CtaSetup&
   cp_async_commit();
 }
 
-// ---------------------------------------------------------------------------
-// Epilogue shared by both engines: merges the warps' (m, l, o) and writes the
-// output (one split) or the split's normalised partial + log2-sum-exp.
-// s_m/s_l: [NWARPS][GP]; s_o: [NWARPS][GP][HD]; s_w: [NWARPS][GP]; s_L: [GP].
-template <int HD, int NWARPS, int GP>
-__device__ __forceinline__ void combine_and_store(const DecodeParams& p, const CtaSetup& c,
-                                                  float* s_m, float* s_l, float* s_o,
-                                                  float* s_w, float* s_L) {
-  const int G = p.group;
-  __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    float M = -CUDART_INF_F;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) M = fmaxf(M, s_m[w * GP + h]);
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) {
-      const float mw = s_m[w * GP + h];
-      const float wt = (mw == -CUDART_INF_F) ? 0.f : exp2f(mw - M);
-      s_w[w * GP + h] = wt;
-      L += wt * s_l[w * GP + h];
-    }
-    s_L[h] = L;
-    if (!p.direct && threadIdx.x < G) {
-      const size_t r = ((size_t)c.seq * p.num_q_heads + (size_t)c.kvh * G + h) * p.ws_slots +
-                       p.ws_base + c.split;
-      p.ws_lse[r] = (L > 0.f) ? M + log2f(L) : -CUDART_INF_F;
-    }
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < G * HD; idx += NWARPS * kWarp) {
-    const int h = idx / HD, d = idx % HD;
-    const float L = s_L[h];
-    float O = 0.f;
-#pragma unroll
-    for (int w = 0; w < NWARPS; ++w) O += s_w[w * GP + h] * s_o[(w * GP + h) * HD + d];
-    const float val = (L > 0.f) ? O / L : 0.f;
-    const size_t qh = (size_t)c.kvh * G + h;
-    if (p.direct) {
-      const size_t o = ((size_t)c.seq * p.num_q_heads + qh) * HD + d;
-      if (p.out_f32)
-        static_cast<float*>(p.out)[o] = val;
-      else
-        static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(val);
-    } else {
-      const size_t o =
-          (((size_t)c.seq * p.num_q_heads + qh) * p.ws_slots + p.ws_base + c.split) * HD + d;
-      p.ws_o[o] = val;
-    }
-  }
-}
-
-// Writes zeros for a sequence with nothing to attend (only the split-0 CTA of
-// a direct launch; the merge kernel covers the other cases).
-template <int HD>
-__device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup& c) {
-  if (!p.direct || c.split != 0) return;
-  const int G = p.group;
-  for (int idx = threadIdx.x; idx < G * HD; idx += blockDim.x) {
-    const int h = idx / HD, d = idx % HD;
-    const size_t o = ((size_t)c.seq * p.num_q_heads + (size_t)c.kvh * G + h) * HD + d;
-    if (p.out_f32)
-      static_cast<float*>(p.out)[o] = 0.f;
-    else
-      static_cast<__nv_bfloat16*>(p.out)[o] = __float2bfloat16_rn(0.f);
-  }
-}
 
 
 // ---------------------------------------------------------------------------
@@ -319,29 +97,24 @@ __device__ __forceinline__ void store_zero(const DecodeParams& p, const CtaSetup
 #ifndef PKV_BF16_STAGES
 #define PKV_BF16_STAGES 2
 #endif
-#ifndef PKV_I8_STAGES
-#define PKV_I8_STAGES 3
-#endif
 
-
-template <int HD, int QM, int NT, int NWARPS, int NSTAGES>
+template <int HD, int NT, int NWARPS, int NSTAGES>
 struct MmaCfg {
-  static constexpr int ELEM = QM != kQuantNone ? 1 : 2;
-  static constexpr int ROWB = HD * ELEM;        // bytes of one token row of one head
-  static constexpr int CH = ROWB / 16;          // 16-byte chunks per row: 4, 8 or 16
+  static constexpr int ROWB = HD * 2;           // bytes of one token row of one head
+  static constexpr int CH = ROWB / 16;          // 16-byte chunks per row: 8 or 16
   static constexpr int RSTEP = kWarp / CH;      // rows one warp-wide copy covers
   static constexpr int PER_LANE = 16 / RSTEP;   // copies per lane per K (or V) tile
   static constexpr int TILE = 16 * ROWB;
-  static constexpr int STAGE = 2 * TILE + (ELEM == 1 ? 128 : 0);
+  static constexpr int STAGE = 2 * TILE;
   static constexpr int RING = NWARPS * NSTAGES * STAGE;
   static constexpr int GP = NT * 8;
   static constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
   static constexpr int BODY = RING > COMB ? RING : COMB;
-  static_assert(CH == 4 || CH == 8 || CH == 16, "rows of 64, 128 or 256 bytes");
+  static_assert(CH == 8 || CH == 16, "rows of 128 or 256 bytes");
 };
 
-// Issues the copies of one 16-token tile (K, V and, for one-byte caches, the
-// 16 per-token scales of each) into a stage, as one commit group.  Full tiles
+// Issues the copies of one 16-token tile (K and V) into a stage, as one
+// commit group.  Full tiles
 // inside one block take the fast path: one block-table lookup, one 64-bit base
 // per lane and fixed per-lane offsets.  Rows outside the sequence or in a bad
 // block are zero-filled.  With AFTER, the stage address is derived from `dep`
@@ -349,7 +122,7 @@ struct MmaCfg {
 template <class Cfg, bool AFTER>
 __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup& c,
                                            const int* s_phys, int tile_t0, uint32_t k_st,
-                                           uint32_t v_st, uint32_t sc_st, int lane,
+                                           uint32_t v_st,
                                            const uint32_t (&soff)[Cfg::PER_LANE],
                                            size_t lane_goff, int lane_row, uint32_t dep) {
   const uint8_t* kb = static_cast<const uint8_t*>(p.k_cache);
@@ -359,11 +132,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
   if constexpr (AFTER) {
     k_st = after_dep(k_st, dep);
     v_st = after_dep(v_st, dep);
-    if constexpr (Cfg::ELEM == 1) sc_st = after_dep(sc_st, dep);
   }
-  // scale row of this lane: lanes 0-15 copy K scales, 16-31 V scales
-  const int srow = lane & 15;
-  const float* ssrc = (lane < 16) ? p.k_scale : p.v_scale;
   if (bs >= 16 && tile_t0 + 16 <= c.t_end) {
     const int phys = s_phys[(tile_t0 >> p.log2_bs) - c.blk0];
     const int n = phys >= 0 ? 16 : 0;
@@ -377,11 +146,6 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
     for (int i = 0; i < Cfg::PER_LANE; ++i) {
       cp_async_16(k_st + soff[i], kp + (size_t)i * step, n);
       cp_async_16(v_st + soff[i], vp + (size_t)i * step, n);
-    }
-    if constexpr (Cfg::ELEM == 1) {
-      const size_t soff_g =
-          phys >= 0 ? ((size_t)phys * p.num_kv_heads + c.kvh) * bs + in_blk + srow : 0;
-      cp_async_4(sc_st + 4 * lane, ssrc + soff_g, phys >= 0 ? 4 : 0);
     }
   } else {
     const size_t lane_col = lane_goff - (size_t)lane_row * tok_stride;  // head + chunk offset
@@ -399,33 +163,20 @@ __device__ __forceinline__ void issue_tile(const DecodeParams& p, const CtaSetup
       cp_async_16(k_st + soff[i], kb + off, n);
       cp_async_16(v_st + soff[i], vb + off, n);
     }
-    if constexpr (Cfg::ELEM == 1) {
-      const int t = tile_t0 + srow;
-      const int phys = phys_of(p, c, s_phys, t);
-      size_t off = 0;
-      int n = 0;
-      if (phys >= 0) {
-        off = ((size_t)phys * p.num_kv_heads + c.kvh) * bs + (t & (bs - 1));
-        n = 4;
-      }
-      cp_async_4(sc_st + 4 * lane, ssrc + off, n);
-    }
   }
   cp_async_commit();
 }
 
-template <int HD, int QM, int NT, int NWARPS, int NSTAGES, bool MHA>
+template <int HD, int NT, int NWARPS, int NSTAGES, bool MHA>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_mma_kernel(const DecodeParams p) {
-  using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
+  pdl_trigger();  // the split merge may be scheduled once every CTA has started
+  using Cfg = MmaCfg<HD, NT, NWARPS, NSTAGES>;
   static_assert(!MHA || NT == 1, "MHA: one q head per kv head");
-  constexpr bool I8 = QM == kQuantI8;
-  constexpr bool F8 = QM == kQuantFp8;
-  constexpr bool Q8 = I8 || F8;         // one-byte codes with per-token scales
   constexpr int KS = HD / 16;           // k-steps of the score mma
   constexpr int MT = HD / 16;           // m-tiles (16 head-dim rows) of the PV mma
-  constexpr int KA = Q8 ? KS / 2 : KS;  // ldmatrix.x4 per K tile
-  constexpr int VA = Q8 ? MT / 2 : MT;  // ldmatrix.x4 per V tile
+  constexpr int KA = KS;                // ldmatrix.x4 per K tile
+  constexpr int VA = MT;                // ldmatrix.x4 per V tile
   constexpr int GP = Cfg::GP;
   constexpr int CH = Cfg::CH;
 
@@ -434,7 +185,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   uint8_t* ring = smem + p.phys_bytes;
 
   long long new_slot;
-  const uint4 new_rows = fused_prefetch<HD, QM>(p, &new_slot);
+  const uint4 new_rows = fused_prefetch<HD, kQuantNone>(p, &new_slot);
   const CtaSetup c = cta_setup(p, s_phys);
   if (!c.active) {
     if (c.split == 0) {
@@ -447,7 +198,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     }
     return;
   }
-  fused_commit<HD, QM, NWARPS>(p, c, s_phys, new_rows, new_slot);  // before any cache read
+  fused_commit<HD, kQuantNone, NWARPS>(p, c, s_phys, new_rows, new_slot);  // before any cache read
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int g = lane >> 2, t4 = lane & 3;
   const int G = p.group;
@@ -465,17 +216,8 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         uint32_t b0 = 0, b1 = 0;
         if (h < G) {
           const __nv_bfloat16* qr = qb + (size_t)h * HD;
-          if constexpr (!Q8) {
-            b0 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4);
-            b1 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4 + 8);
-          } else {
-            // k-slot order of a one-byte-code chunk: slots 2t,2t+1 <- d 16c+4t+{0,1},
-            // slots 2t+8,2t+9 <- d 16c+4t+{2,3}
-            const uint2 raw = *reinterpret_cast<const uint2*>(qr + 16 * ks + 4 * t4);
-            const float2 lo = unpack_bf16(raw.x), hi = unpack_bf16(raw.y);
-            b0 = pack_f16(lo.x, lo.y);
-            b1 = pack_f16(hi.x, hi.y);
-          }
+          b0 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4);
+          b1 = *reinterpret_cast<const uint32_t*>(qr + 16 * ks + 2 * t4 + 8);
         }
         qf[ks][nt][0] = b0;
         qf[ks][nt][1] = b1;
@@ -483,34 +225,14 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     }
   }
 
-  // INT8: the tensor core sees code + 1152 instead of code (see
-  // i8pair_to_f16x2_biased), so every score carries 1152 * sum_d q[h][d]; qbias
-  // holds that term for this thread's two head columns 2*t4 and 2*t4 + 1.
-  float qbias[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    float mine = 0.f;  // partial sum over this lane's k-slots of head nt*8 + g
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const float2 a = unpack_f16(qf[ks][nt][0]), b = unpack_f16(qf[ks][nt][1]);
-      mine += (a.x + a.y) + (b.x + b.y);
-    }
-    mine += __shfl_xor_sync(0xffffffffu, mine, 1);
-    mine += __shfl_xor_sync(0xffffffffu, mine, 2);
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-      qbias[nt][j] = I8 ? 1152.f * __shfl_sync(0xffffffffu, mine, (2 * t4 + j) * 4) : 0.f;
-  }
-
   float o[MT][NT][4];
-  float m_run[NT][2], l_run[NT][2], p_run[NT][2];
+  float m_run[NT][2], l_run[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       m_run[nt][j] = -CUDART_INF_F;
       l_run[nt][j] = 0.f;
-      p_run[nt][j] = 0.f;  // INT8: sum of the P fed to the PV mma (for its 1152 bias)
     }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
@@ -539,8 +261,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   for (int i = 0; i < KA; ++i) koff[i] = (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16;
 #pragma unroll
   for (int i = 0; i < VA; ++i)
-    voff[i] = Q8 ? (uint32_t)swz<CH>(lm_row_a, 2 * i + lm_ch_a) * 16
-                 : (uint32_t)swz<CH>(lm_row_v, 2 * i + lm_ch_v) * 16;
+    voff[i] = (uint32_t)swz<CH>(lm_row_v, 2 * i + lm_ch_v) * 16;
 
   const uint32_t my_ring = smem_u32(ring) + (uint32_t)(warp * NSTAGES * Cfg::STAGE);
   const int ntiles = (c.t_end - c.t_begin + 15) >> 4;
@@ -551,8 +272,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     const uint32_t st = my_ring + (uint32_t)(i * Cfg::STAGE);
     if (i < my_n)
       issue_tile<Cfg, false>(p, c, s_phys, c.t_begin + (warp + i * NWARPS) * 16, st,
-                             st + Cfg::TILE, st + 2 * Cfg::TILE, lane, soff, lane_goff, lane_row,
-                             0u);
+                             st + Cfg::TILE, soff, lane_goff, lane_row, 0u);
     else
       cp_async_commit();
   }
@@ -573,17 +293,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
     for (int a = 0; a < VA; ++a)
       ldmatrix_x4_trans(vS + voff[a], vf[a][0], vf[a][1], vf[a][2], vf[a][3]);
-    float ska = 0.f, skb = 0.f, sva = 0.f, svb = 0.f;
     uint32_t dep = 0;
-    if constexpr (Q8) {
-      float mine;
-      asm volatile("ld.shared.f32 %0, [%1];\n" : "=f"(mine) : "r"(vS + Cfg::TILE + 4 * lane));
-      ska = __shfl_sync(0xffffffffu, mine, g);
-      skb = __shfl_sync(0xffffffffu, mine, g + 8);
-      sva = __shfl_sync(0xffffffffu, mine, 16 + g);
-      svb = __shfl_sync(0xffffffffu, mine, 24 + g);
-      dep = __float_as_uint(mine);
-    }
     // one register of each ldmatrix: an ldmatrix completes all of its registers at once
 #pragma unroll
     for (int a = 0; a < KA; ++a) dep ^= kf[a][0];
@@ -596,8 +306,8 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     {
       const int ii = i + NSTAGES;
       if (ii < my_n)
-        issue_tile<Cfg, true>(p, c, s_phys, tile_t0 + NSTAGES * NWARPS * 16, kS, vS,
-                              vS + Cfg::TILE, lane, soff, lane_goff, lane_row, dep);
+        issue_tile<Cfg, true>(p, c, s_phys, tile_t0 + NSTAGES * NWARPS * 16, kS, vS, soff,
+                              lane_goff, lane_row, dep);
       else
         cp_async_commit();
     }
@@ -609,75 +319,22 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[nt][q] = acc2[nt][q] = 0.f;
-    if constexpr (!Q8) {
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
+    for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if (ks & 1)
-            mma_bf16(acc2[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
-                     qf[ks][nt][1]);
-          else
-            mma_bf16(acc[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
-                     qf[ks][nt][1]);
-        }
-      }
-    } else if constexpr (F8) {
-#pragma unroll
-      for (int kp = 0; kp < KS / 2; ++kp) {
-        // kf[kp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1); bytes of a
-        // register are d 4t..4t+3 -> slots (2t, 2t+1) (its low half) and
-        // (2t+8, 2t+9) (its high half), so each half converts as it is
-        const uint32_t top[2] = {kf[kp][0], kf[kp][2]};
-        const uint32_t bot[2] = {kf[kp][1], kf[kp][3]};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = e4m3half_to_f16x2<true>(top[h]);
-          const uint32_t a2 = e4m3half_to_f16x2<false>(top[h]);
-          const uint32_t a1 = e4m3half_to_f16x2<true>(bot[h]);
-          const uint32_t a3 = e4m3half_to_f16x2<false>(bot[h]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (h)
-              mma_f16(acc2[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
-            else
-              mma_f16(acc[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
-          }
-        }
-      }
-    } else {
-#pragma unroll
-      for (int kp = 0; kp < KS / 2; ++kp) {
-        // kf[kp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1)
-        const uint32_t top[2] = {kf[kp][0] ^ 0x80808080u, kf[kp][2] ^ 0x80808080u};
-        const uint32_t bot[2] = {kf[kp][1] ^ 0x80808080u, kf[kp][3] ^ 0x80808080u};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = i8pair_to_f16x2_biased<0x4140>(top[h]);
-          const uint32_t a2 = i8pair_to_f16x2_biased<0x4342>(top[h]);
-          const uint32_t a1 = i8pair_to_f16x2_biased<0x4140>(bot[h]);
-          const uint32_t a3 = i8pair_to_f16x2_biased<0x4342>(bot[h]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            if (h)
-              mma_f16(acc2[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
-            else
-              mma_f16(acc[nt], a0, a1, a2, a3, qf[2 * kp + h][nt][0], qf[2 * kp + h][nt][1]);
-          }
-        }
+      for (int nt = 0; nt < NT; ++nt) {
+        if (ks & 1)
+          mma_bf16(acc2[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
+                   qf[ks][nt][1]);
+        else
+          mma_bf16(acc[nt], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][nt][0],
+                   qf[ks][nt][1]);
       }
     }
 
     // ---- mask, scale, online softmax (tokens g, g+8; heads 2t4, 2t4+1)
     const bool va = (mask >> g) & 1u, vb = (mask >> (g + 8)) & 1u;
-    float fa = p.scale_log2, fb = p.scale_log2;
-    float pva = 1.f, pvb = 1.f;
-    if constexpr (Q8) {
-      fa = va ? fa * fast_rcp(ska) : 0.f;
-      fb = vb ? fb * fast_rcp(skb) : 0.f;
-      pva = va ? fast_rcp(sva) : 0.f;
-      pvb = vb ? fast_rcp(svb) : 0.f;
-    }
+    const float fa = p.scale_log2, fb = p.scale_log2;
     uint32_t bh[NT][2], bl[NT][2];
     float alpha[NT][2];
     bool rescale = false;
@@ -692,10 +349,8 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
           continue;
         }
         // scores of head 2*t4 + jj for tokens g (sa) and g + 8 (sb)
-        const float sa =
-            va ? ((acc[nt][jj] + acc2[nt][jj]) - qbias[nt][jj]) * fa : -CUDART_INF_F;
-        const float sb =
-            vb ? ((acc[nt][jj + 2] + acc2[nt][jj + 2]) - qbias[nt][jj]) * fb : -CUDART_INF_F;
+        const float sa = va ? (acc[nt][jj] + acc2[nt][jj]) * fa : -CUDART_INF_F;
+        const float sb = vb ? (acc[nt][jj + 2] + acc2[nt][jj + 2]) * fb : -CUDART_INF_F;
         float mx = fmaxf(sa, sb);
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -710,24 +365,13 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         alpha[nt][jj] = a;
         rescale |= (a != 1.f);
       }
-      const float q0 = pr[0] * pva, q1 = pr[1] * pva, q2 = pr[2] * pvb, q3 = pr[3] * pvb;
-      if constexpr (!Q8) {
-        const uint32_t h01 = pack_bf16(q0, q1), h23 = pack_bf16(q2, q3);
-        const float2 f01 = unpack_bf16(h01), f23 = unpack_bf16(h23);
-        bh[nt][0] = movmatrix_trans(h01);
-        bh[nt][1] = movmatrix_trans(h23);
-        bl[nt][0] = movmatrix_trans(pack_bf16(q0 - f01.x, q1 - f01.y));
-        bl[nt][1] = movmatrix_trans(pack_bf16(q2 - f23.x, q3 - f23.y));
-      } else {
-        const uint32_t h01 = pack_f16(q0, q1), h23 = pack_f16(q2, q3);
-        if constexpr (I8) {  // the P the tensor core sees, for the 1152 bias
-          const float2 f01 = unpack_f16(h01), f23 = unpack_f16(h23);
-          p_run[nt][0] = p_run[nt][0] * alpha[nt][0] + (f01.x + f23.x);
-          p_run[nt][1] = p_run[nt][1] * alpha[nt][1] + (f01.y + f23.y);
-        }
-        bh[nt][0] = movmatrix_trans(h01);
-        bh[nt][1] = movmatrix_trans(h23);
-      }
+      const float q0 = pr[0], q1 = pr[1], q2 = pr[2], q3 = pr[3];
+      const uint32_t h01 = pack_bf16(q0, q1), h23 = pack_bf16(q2, q3);
+      const float2 f01 = unpack_bf16(h01), f23 = unpack_bf16(h23);
+      bh[nt][0] = movmatrix_trans(h01);
+      bh[nt][1] = movmatrix_trans(h23);
+      bl[nt][0] = movmatrix_trans(pack_bf16(q0 - f01.x, q1 - f01.y));
+      bl[nt][1] = movmatrix_trans(pack_bf16(q2 - f23.x, q3 - f23.y));
     }
     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -741,75 +385,17 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
         }
     }
 
-    // ---- O^T[d][head] += V^T * P^T
-    if constexpr (!Q8) {
+    // ---- O^T[d][head] += V^T * P^T (P as bf16 hi + lo)
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bh[nt][0], bh[nt][1]);
-          mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bl[nt][0], bl[nt][1]);
-        }
-      }
-    } else if constexpr (F8) {
-#pragma unroll
-      for (int mp = 0; mp < MT / 2; ++mp) {
-        // vf[mp] transposed: a register holds bytes (t 2t, d 2g) (2t, 2g+1)
-        // (2t+1, 2g) (2t+1, 2g+1); rows m <-> d as in the INT8 case
-        const uint32_t top[2] = {vf[mp][0], vf[mp][2]};
-        const uint32_t bot[2] = {vf[mp][1], vf[mp][3]};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = e4m3pair_to_f16x2<0x0020>(top[h]);
-          const uint32_t a1 = e4m3pair_to_f16x2<0x0031>(top[h]);
-          const uint32_t a2 = e4m3pair_to_f16x2<0x0020>(bot[h]);
-          const uint32_t a3 = e4m3pair_to_f16x2<0x0031>(bot[h]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-          }
-        }
-      }
-    } else {
-#pragma unroll
-      for (int mp = 0; mp < MT / 2; ++mp) {
-        // vf[mp]: (rows 0-7, c) (rows 8-15, c) (0-7, c+1) (8-15, c+1), transposed
-        const uint32_t top[2] = {vf[mp][0] ^ 0x80808080u, vf[mp][2] ^ 0x80808080u};
-        const uint32_t bot[2] = {vf[mp][1] ^ 0x80808080u, vf[mp][3] ^ 0x80808080u};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // rows m <-> d: m = g -> 16c + 2g, m = g + 8 -> 16c + 2g + 1
-          const uint32_t a0 = i8pair_to_f16x2_biased<0x4240>(top[h]);
-          const uint32_t a1 = i8pair_to_f16x2_biased<0x4341>(top[h]);
-          const uint32_t a2 = i8pair_to_f16x2_biased<0x4240>(bot[h]);
-          const uint32_t a3 = i8pair_to_f16x2_biased<0x4341>(bot[h]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_f16(o[2 * mp + h][nt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-          }
-        }
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bh[nt][0], bh[nt][1]);
+        mma_bf16(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bl[nt][0], bl[nt][1]);
       }
     }
   }
   cp_async_wait<0>();
-
-  if constexpr (I8) {
-    // O carries 1152 * sum_t P[t][h] from the biased V codes: remove it.
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float ps = p_run[nt][j];
-        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
-        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          o[mt][nt][j] -= 1152.f * ps;
-          o[mt][nt][j + 2] -= 1152.f * ps;
-        }
-      }
-  }
 
   // ---- per-warp final state -> smem (the ring is reused: wait for every warp)
 #pragma unroll
@@ -845,7 +431,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
       for (int j = 0; j < 4; ++j) {
         const int m = g + (j >> 1) * 8;  // fragment row
         const int h = nt * 8 + 2 * t4 + (j & 1);
-        const int d = Q8 ? 16 * mt + (m < 8 ? 2 * m : 2 * (m - 8) + 1) : 16 * mt + m;
+        const int d = 16 * mt + m;
         s_o[(warp * GP + h) * HD + d] = o[mt][nt][j];
       }
   combine_and_store<HD, NWARPS, GP>(p, c, s_m, s_l, s_o, s_w, s_L);
@@ -858,6 +444,7 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 template <int HD, int NWARPS, int NSTAGES>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_simt_kernel(const DecodeParams p) {
+  pdl_trigger();
   constexpr int ELEM = 4;
   constexpr int ROWB = HD * ELEM;
   constexpr int CH = ROWB / 16;
@@ -1033,6 +620,7 @@ constexpr int kMergeBatch = 8;  // partial rows in flight per lane
 
 template <int HD>
 __global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeParams p) {
+  pdl_wait();  // the decode grid's partials are complete and visible past this point
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x % kWarp;
   const int qh = blockIdx.x * kMergeWarps + warp, seq = blockIdx.y;
   if (qh >= p.num_q_heads) return;
@@ -1101,49 +689,11 @@ __global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeP
 
 namespace {
 
-// Raises a kernel's dynamic shared-memory limit once per (device, kernel) to
-// the device's opt-in maximum; later launches skip the runtime call.  The
-// cached limit is per kernel (the kernel is the template argument).  Racing
-// first calls from several host threads set the same value.
-constexpr int kMaxDevices = 64;
-
-template <auto Kernel>
-cudaError_t prepare(int smem) {
-  static std::atomic<int> limit[kMaxDevices];  // raised limit per device, 0 = not yet
-  if (smem <= 48 * 1024) return cudaSuccess;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const bool cached = dev >= 0 && dev < kMaxDevices;
-  if (cached) {
-    const int l = limit[dev].load(std::memory_order_acquire);
-    if (l > 0) return smem <= l ? cudaSuccess : cudaErrorInvalidValue;
-  }
-  int optin = 0;
-  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  if (e != cudaSuccess) return e;
-  if (smem > optin) return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess && cached) limit[dev].store(optin, std::memory_order_release);
-  return e;
-}
-
-// Shared memory of one sm_100 SM, and the part the hardware reserves per CTA.
-constexpr int kSmemPerSm = 228 * 1024, kSmemPerCta = 1024;
-// A dynamic shared-memory request above which at most three CTAs fit an SM.
-constexpr int kThreeCtaSmem = kSmemPerSm / 4 - kSmemPerCta + 16;
-
-template <int HD, int QM, int NT, int NWARPS, int NSTAGES, bool MHA>
+template <int HD, int NT, int NWARPS, int NSTAGES, bool MHA>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = MmaCfg<HD, QM, NT, NWARPS, NSTAGES>;
-  int smem = p.phys_bytes + Cfg::BODY;
-  // The one-byte MHA kernels at head_dim 128 fit four CTAs per SM by
-  // registers, the other one-byte kernels three.  Held to three as well, the
-  // FP8 13B workload ran 3% faster (INT8 within 1%), and the split planner's
-  // occupancy figure (taken from the general kernel) stays exact.
-  if constexpr (MHA && QM != kQuantNone && HD == 128)
-    smem = smem > kThreeCtaSmem ? smem : kThreeCtaSmem;
-  constexpr auto k = decode_mma_kernel<HD, QM, NT, NWARPS, NSTAGES, MHA>;
+  using Cfg = MmaCfg<HD, NT, NWARPS, NSTAGES>;
+  const int smem = p.phys_bytes + Cfg::BODY;
+  constexpr auto k = decode_mma_kernel<HD, NT, NWARPS, NSTAGES, MHA>;
   cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
@@ -1188,23 +738,19 @@ int occupancy(int threads, int smem) {
 
 constexpr int kTypicalPhysBytes = 1024;  // block-table slice of a typical split
 
-template <int HD, int QM>
+template <int HD>
 int mma_occupancy() {
-  constexpr int NS = QM != kQuantNone ? PKV_I8_STAGES : PKV_BF16_STAGES;
-  using Cfg = MmaCfg<HD, QM, 1, kMW, NS>;
-  return occupancy<decode_mma_kernel<HD, QM, 1, kMW, NS, false>>(kMW * kWarp,
-                                                          kTypicalPhysBytes + Cfg::BODY);
+  constexpr int NS = PKV_BF16_STAGES;
+  using Cfg = MmaCfg<HD, 1, kMW, NS>;
+  return occupancy<decode_mma_kernel<HD, 1, kMW, NS, false>>(kMW * kWarp,
+                                                       kTypicalPhysBytes + Cfg::BODY);
 }
 
 }  // namespace
 
 int decode_ctas_per_sm_hint(pkv_dtype cache_dt, int head_dim) {
-  if (cache_dt == PKV_BF16) return head_dim == 128 ? mma_occupancy<128, kQuantNone>()
-                                                   : mma_occupancy<64, kQuantNone>();
-  if (cache_dt == PKV_I8) return head_dim == 128 ? mma_occupancy<128, kQuantI8>()
-                                                 : mma_occupancy<64, kQuantI8>();
-  if (cache_dt == PKV_FP8) return head_dim == 128 ? mma_occupancy<128, kQuantFp8>()
-                                                  : mma_occupancy<64, kQuantFp8>();
+  if (cache_dt == PKV_BF16) return head_dim == 128 ? mma_occupancy<128>() : mma_occupancy<64>();
+  if (cache_dt == PKV_I8 || cache_dt == PKV_FP8) return decode_q8_ctas_per_sm(cache_dt, head_dim);
   const int smem = kF32Warps * kF32Stages * 2 * 16 * head_dim * 4 + 16 * head_dim * 4 + 1024;
   const int n = kSmemPerSm / (smem + kSmemPerCta);
   return n < 1 ? 1 : n;
@@ -1214,11 +760,11 @@ namespace {
 
 // Picks the q-head tiling: two n-tiles for groups above 8, the MHA form for a
 // group of one, else one n-tile.
-template <int HD, int QM, int NS>
+template <int HD, int NS>
 cudaError_t launch_mma_group(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  if (p.group > 8) return launch_mma<HD, QM, 2, kMW, NS, false>(p, grid, st);
-  if (p.group == 1) return launch_mma<HD, QM, 1, kMW, NS, true>(p, grid, st);
-  return launch_mma<HD, QM, 1, kMW, NS, false>(p, grid, st);
+  if (p.group > 8) return launch_mma<HD, 2, kMW, NS, false>(p, grid, st);
+  if (p.group == 1) return launch_mma<HD, 1, kMW, NS, true>(p, grid, st);
+  return launch_mma<HD, 1, kMW, NS, false>(p, grid, st);
 }
 
 }  // namespace
@@ -1227,24 +773,31 @@ cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_di
                           cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.num_seqs, p.num_splits);
   if (cache_dt == PKV_BF16)
-    return head_dim == 128 ? launch_mma_group<128, kQuantNone, PKV_BF16_STAGES>(p, grid, st)
-                           : launch_mma_group<64, kQuantNone, PKV_BF16_STAGES>(p, grid, st);
-  if (cache_dt == PKV_I8)
-    return head_dim == 128 ? launch_mma_group<128, kQuantI8, PKV_I8_STAGES>(p, grid, st)
-                           : launch_mma_group<64, kQuantI8, PKV_I8_STAGES>(p, grid, st);
-  if (cache_dt == PKV_FP8)
-    return head_dim == 128 ? launch_mma_group<128, kQuantFp8, PKV_I8_STAGES>(p, grid, st)
-                           : launch_mma_group<64, kQuantFp8, PKV_I8_STAGES>(p, grid, st);
+    return head_dim == 128 ? launch_mma_group<128, PKV_BF16_STAGES>(p, grid, st)
+                           : launch_mma_group<64, PKV_BF16_STAGES>(p, grid, st);
+  if (cache_dt == PKV_I8 || cache_dt == PKV_FP8) return launch_decode_q8(p, cache_dt, head_dim, st);
   if (head_dim == 128) return launch_simt<128, kF32Warps, kF32Stages>(p, grid, st);
   return launch_simt<64, kF32Warps, kF32Stages>(p, grid, st);
 }
 
+// The merge is launched with programmatic stream serialization: its CTAs
+// may become resident while the decode grid's last CTAs run (every decode CTA
+// signals at its start), and each waits in pdl_wait for the decode grid to
+// complete, so the launch latency hides behind the decode's tail.
 cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st) {
-  dim3 grid((p.num_q_heads + kMergeWarps - 1) / kMergeWarps, p.num_seqs);
-  if (head_dim == 128)
-    merge_kernel<128><<<grid, kMergeWarps * kWarp, 0, st>>>(p);
-  else
-    merge_kernel<64><<<grid, kMergeWarps * kWarp, 0, st>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.num_q_heads + kMergeWarps - 1) / kMergeWarps, p.num_seqs);
+  cfg.blockDim = dim3(kMergeWarps * kWarp);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = head_dim == 128 ? cudaLaunchKernelEx(&cfg, merge_kernel<128>, p)
+                                  : cudaLaunchKernelEx(&cfg, merge_kernel<64>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -55,8 +55,16 @@ constexpr int kMaxPrefixChunk = 8192;  // prefix tokens per slice at most
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
                           cudaStream_t st);
+// One-byte caches (INT8, FP8): the engine of decode_q8.cu, and how many of its
+// CTAs fit one SM.
+cudaError_t launch_decode_q8(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
+                             cudaStream_t st);
+int decode_q8_ctas_per_sm(pkv_dtype cache_dt, int head_dim);
+// behind_decode: the pass is launched right after the suffix decode of the
+// same call, with programmatic stream serialization (it may start while that
+// decode's last CTAs run, and completes only after that decode).
 cudaError_t launch_prefix(const DecodeParams& p, const PrefixParams& pp, int head_dim,
-                          cudaStream_t st);
+                          bool behind_decode, cudaStream_t st);
 // CTAs of rows per KV head in the shared-prefix pass (128 / group sequences each).
 int prefix_row_groups(int num_seqs, int group);
 cudaError_t launch_merge(const DecodeParams& p, int head_dim, cudaStream_t st);

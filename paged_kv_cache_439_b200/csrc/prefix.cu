@@ -265,6 +265,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v) {
   using Cfg = TcCfg<HD>;
+  pdl_trigger();  // the split merge may be scheduled once every CTA has started
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
@@ -652,6 +653,10 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
                  "r"(Cfg::TMEM_COLS)
                  : "memory");
   }
+  // Launched behind the suffix decode (see launch_prefix), this grid may start
+  // before that one ends; it completes only after it, so the merge, which
+  // waits for this grid, also sees every suffix partial.
+  pdl_wait();
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -709,7 +714,7 @@ cudaError_t prepare(int dev) {
 }
 
 template <int HD>
-cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, cudaStream_t st) {
+cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, bool behind, cudaStream_t st) {
   const int smem = smem_bytes<HD>(pp);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -727,8 +732,18 @@ cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, cudaStream_t s
   if (e == cudaSuccess)
     e = bf16_map(&tv, p.v_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.num_kv_heads, pp.prefix_splits, (p.num_seqs + spc - 1) / spc);
-  prefix_kernel<HD><<<grid, kTcThreads, smem, st>>>(p, pp, tq, tk, tv);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.num_kv_heads, pp.prefix_splits, (p.num_seqs + spc - 1) / spc);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = behind ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, prefix_kernel<HD>, p, pp, tq, tk, tv);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -740,9 +755,9 @@ int prefix_row_groups(int num_seqs, int group) {
 }
 
 cudaError_t launch_prefix(const DecodeParams& p, const PrefixParams& pp, int head_dim,
-                          cudaStream_t st) {
-  if (head_dim == 128) return launch<128>(p, pp, st);
-  return launch<64>(p, pp, st);
+                          bool behind_decode, cudaStream_t st) {
+  if (head_dim == 128) return launch<128>(p, pp, behind_decode, st);
+  return launch<64>(p, pp, behind_decode, st);
 }
 
 }  // namespace pkv

@@ -46,9 +46,11 @@ def test_append_bit_exact(cache_dtype, d, bs):
     assert g.flags() == 0
 
 
-def test_append_int8_full_13b_bulk():
-    """Bulk fill of the Llama-2-13B-shaped INT8 workload (65,504 pre-fill tokens)."""
-    wl = make_workload("llama2-13b-int8")
+@pytest.mark.parametrize("kv", ["i8", "fp8"])
+def test_append_int8_full_13b_bulk(kv):
+    """Bulk fill of the Llama-2-13B-shaped workload (65,504 pre-fill tokens),
+    INT8 and FP8 caches, bit for bit."""
+    wl = make_workload("llama2-13b-int8", cache_dtype=kv)
     g = GpuCache(wl).fill()
     o = OracleCache(wl).fill()
     torch.cuda.synchronize()
@@ -163,8 +165,9 @@ def test_splits_agree():
 
 # ---------------------------------------------------------------- edges
 
-def test_empty_and_single_token_contexts():
-    wl = _wl("bf16", 8, 2, 128, 16, lens=[0, 1, 0, 2, 16])
+@pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8"])
+def test_empty_and_single_token_contexts(cache_dtype):
+    wl = _wl(cache_dtype, 8, 2, 128, 16, lens=[0, 1, 0, 2, 16])
     g = GpuCache(wl).fill()
     ref = OracleCache(wl).fill().decode()
     for splits in (0, 1, 2):
@@ -173,9 +176,10 @@ def test_empty_and_single_token_contexts():
         assert_close(out, ref, tol_for(wl), f"edges s={splits}")
 
 
-def test_padded_table_entries_never_read():
+@pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8"])
+def test_padded_table_entries_never_read(cache_dtype):
     # entries past each sequence's last block point outside the pool
-    wl = _wl("bf16", 8, 2, 64, 16, lens=[5, 40], pad_entry=10**6, extra_table_cols=3)
+    wl = _wl(cache_dtype, 8, 2, 64, 16, lens=[5, 40], pad_entry=10**6, extra_table_cols=3)
     g = GpuCache(wl).fill()
     ref = OracleCache(wl).fill().decode(block_tables=torch.where(
         wl.block_tables >= wl.num_blocks, torch.full_like(wl.block_tables, -1), wl.block_tables))
@@ -183,8 +187,9 @@ def test_padded_table_entries_never_read():
     assert g.flags() == 0
 
 
-def test_bad_block_sets_flag_and_is_skipped():
-    wl = _wl("bf16", 8, 2, 64, 16, lens=[64, 40])
+@pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8"])
+def test_bad_block_sets_flag_and_is_skipped(cache_dtype):
+    wl = _wl(cache_dtype, 8, 2, 64, 16, lens=[64, 40])
     g = GpuCache(wl).fill()
     bt = wl.block_tables.clone()
     bt[0, 1] = wl.num_blocks + 3          # tokens 16..31 of sequence 0 are unreachable
@@ -240,3 +245,17 @@ def test_full_workload_parity(name, bs, kv):
     r = assert_close(out, ref, tol_for(wl), name)
     assert g.flags() == 0
     print(f"{name} bs={wl.block_size}: max_abs={r['max_abs']:.2e} max_rel={r['max_rel']:.2e}")
+
+
+@pytest.mark.parametrize("cache_dtype", ["i8", "fp8", "bf16"])
+def test_query_spread_over_many_binades(cache_dtype):
+    """q elements spread over 24 binades (so they do not share one exponent):
+    the one-byte engines' score paths stay within the stated tolerance."""
+    wl = _wl(cache_dtype, 8, 8, 128, 16, lens=[33, 700, 2048], outlier_prob=0.01)
+    gen = torch.Generator().manual_seed(5)
+    mag = torch.pow(2.0, torch.randint(-20, 5, wl.q.shape, generator=gen).float())
+    wl.q = (torch.randn(wl.q.shape, generator=gen) * mag).to(wl.q.dtype)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1, 3):
+        assert_close(g.decode(num_splits=splits), ref, tol_for(wl), f"spread s={splits}")
