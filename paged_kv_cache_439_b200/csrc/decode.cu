@@ -438,20 +438,22 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 }
 
 // ---------------------------------------------------------------------------
-// simt engine: fp32 caches, q in fp32 or bf16.  Lanes l and l+16 share token
+// simt engine: fp32 caches (ELEM 4; q in fp32 or bf16), or bf16 caches
+// (ELEM 2) where the tensor cores are not used.  Lanes l and l+16 share token
 // l%16, each summing half of head_dim; the PV update gives lane l the head_dim
-// columns l, l+32, ...
-template <int HD, int NWARPS, int NSTAGES>
+// columns l, l+32, ... (fp32) or the pairs 2l, 2l+1, 2l+64, 2l+65 (bf16).  GP
+// (a power of two, at least the group) bounds the q heads held per thread.
+template <int HD, int NWARPS, int NSTAGES, int ELEM, int GP>
 __global__ void __launch_bounds__(NWARPS * kWarp)
     decode_simt_kernel(const DecodeParams p) {
   pdl_trigger();
-  constexpr int ELEM = 4;
+  static_assert(ELEM == 4 || ELEM == 2, "fp32 or bf16 cache rows");
   constexpr int ROWB = HD * ELEM;
   constexpr int CH = ROWB / 16;
   constexpr int TILE_B = 16 * ROWB;
   constexpr int STAGE_B = 2 * TILE_B;
-  constexpr int GP = 16;
   constexpr int DJ = HD / kWarp;
+  constexpr int EPC = 16 / ELEM;  // elements per 16-byte chunk
 
   extern __shared__ __align__(128) uint8_t smem[];
   int* s_phys = reinterpret_cast<int*>(smem);
@@ -525,15 +527,33 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll
     for (int cc = 0; cc < CH / 2; ++cc) {
       const int ch = hf * (CH / 2) + cc;
-      const float4 kv = *reinterpret_cast<const float4*>(kt + swz<CH>(tr, ch) * 16);
+      const uint4 raw = *reinterpret_cast<const uint4*>(kt + swz<CH>(tr, ch) * 16);
+      float kv[EPC];
+      if constexpr (ELEM == 4) {
+        kv[0] = __uint_as_float(raw.x);
+        kv[1] = __uint_as_float(raw.y);
+        kv[2] = __uint_as_float(raw.z);
+        kv[3] = __uint_as_float(raw.w);
+      } else {
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = unpack_bf16(w[k]);
+          kv[2 * k] = f.x;
+          kv[2 * k + 1] = f.y;
+        }
+      }
 #pragma unroll
       for (int h = 0; h < GP; ++h) {
         if (h < G) {
-          const float4 qv = *reinterpret_cast<const float4*>(s_q + h * HD + ch * 4);
-          s[h] = fmaf(qv.x, kv.x, s[h]);
-          s[h] = fmaf(qv.y, kv.y, s[h]);
-          s[h] = fmaf(qv.z, kv.z, s[h]);
-          s[h] = fmaf(qv.w, kv.w, s[h]);
+#pragma unroll
+          for (int e4 = 0; e4 < EPC; e4 += 4) {
+            const float4 qv = *reinterpret_cast<const float4*>(s_q + h * HD + ch * EPC + e4);
+            s[h] = fmaf(qv.x, kv[e4], s[h]);
+            s[h] = fmaf(qv.y, kv[e4 + 1], s[h]);
+            s[h] = fmaf(qv.z, kv[e4 + 2], s[h]);
+            s[h] = fmaf(qv.w, kv[e4 + 3], s[h]);
+          }
         }
       }
     }
@@ -561,10 +581,21 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
 #pragma unroll 4
     for (int t = 0; t < 16; ++t) {
       float vv[DJ];
+      if constexpr (ELEM == 4) {
 #pragma unroll
-      for (int j = 0; j < DJ; ++j) {
-        const int e = lane + kWarp * j;
-        vv[j] = *reinterpret_cast<const float*>(vt + swz<CH>(t, e >> 2) * 16 + (e & 3) * 4);
+        for (int j = 0; j < DJ; ++j) {
+          const int e = lane + kWarp * j;
+          vv[j] = *reinterpret_cast<const float*>(vt + swz<CH>(t, e >> 2) * 16 + (e & 3) * 4);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < DJ / 2; ++j) {
+          const int e = 2 * lane + 2 * kWarp * j;  // column pair e, e + 1
+          const float2 f = unpack_bf16(*reinterpret_cast<const uint32_t*>(
+              vt + swz<CH>(t, e >> 3) * 16 + (e & 7) * 2));
+          vv[2 * j] = f.x;
+          vv[2 * j + 1] = f.y;
+        }
       }
 #pragma unroll
       for (int h = 0; h < GP; ++h) {
@@ -602,7 +633,10 @@ __global__ void __launch_bounds__(NWARPS * kWarp)
   for (int h = 0; h < GP; ++h)
     if (h < G)
 #pragma unroll
-      for (int j = 0; j < DJ; ++j) s_o[(warp * GP + h) * HD + lane + kWarp * j] = o[h][j];
+      for (int j = 0; j < DJ; ++j) {
+        const int d = ELEM == 4 ? lane + kWarp * j : 2 * lane + 2 * kWarp * (j >> 1) + (j & 1);
+        s_o[(warp * GP + h) * HD + d] = o[h][j];
+      }
   combine_and_store<HD, NWARPS, GP>(p, c, s_m, s_l, s_o, s_w, s_L);
 }
 
@@ -700,14 +734,13 @@ cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-template <int HD, int NWARPS, int NSTAGES>
+template <int HD, int NWARPS, int NSTAGES, int ELEM = 4, int GP = 16>
 cudaError_t launch_simt(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  constexpr int STAGE_B = 2 * 16 * HD * 4;
+  constexpr int STAGE_B = 2 * 16 * HD * ELEM;
   constexpr int RING = NWARPS * NSTAGES * STAGE_B;
-  constexpr int GP = 16;
   constexpr int COMB = (3 * NWARPS * GP + GP + NWARPS * GP * HD) * 4;
   const int smem = p.phys_bytes + GP * HD * 4 + (RING > COMB ? RING : COMB);
-  constexpr auto k = decode_simt_kernel<HD, NWARPS, NSTAGES>;
+  constexpr auto k = decode_simt_kernel<HD, NWARPS, NSTAGES, ELEM, GP>;
   cudaError_t e = prepare<k>(smem);
   if (e != cudaSuccess) return e;
   k<<<grid, NWARPS * kWarp, smem, st>>>(p);
@@ -769,9 +802,29 @@ cudaError_t launch_mma_group(const DecodeParams& p, dim3 grid, cudaStream_t st) 
 
 }  // namespace
 
+// bf16 caches on the SIMT engine instead of the tensor cores, for groups below
+// this value (0: never).  The tensor-core engine is the default at every group
+// size: measured against this SIMT form at groups 1 and 4 it was faster (the
+// figures are in the project's design notes); the switch exists to repeat that
+// comparison.
+#ifndef PKV_SIMT_BELOW_GROUP
+#define PKV_SIMT_BELOW_GROUP 0
+#endif
+
+template <int HD>
+cudaError_t launch_simt_bf16(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  if (p.group <= 1) return launch_simt<HD, kF32Warps, kF32Stages, 2, 1>(p, grid, st);
+  if (p.group <= 2) return launch_simt<HD, kF32Warps, kF32Stages, 2, 2>(p, grid, st);
+  if (p.group <= 4) return launch_simt<HD, kF32Warps, kF32Stages, 2, 4>(p, grid, st);
+  if (p.group <= 8) return launch_simt<HD, kF32Warps, kF32Stages, 2, 8>(p, grid, st);
+  return launch_simt<HD, kF32Warps, kF32Stages, 2, 16>(p, grid, st);
+}
+
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,
                           cudaStream_t st) {
   dim3 grid(p.num_kv_heads, p.num_seqs, p.num_splits);
+  if (cache_dt == PKV_BF16 && p.group < PKV_SIMT_BELOW_GROUP && p.new_k == nullptr)
+    return head_dim == 128 ? launch_simt_bf16<128>(p, grid, st) : launch_simt_bf16<64>(p, grid, st);
   if (cache_dt == PKV_BF16)
     return head_dim == 128 ? launch_mma_group<128, PKV_BF16_STAGES>(p, grid, st)
                            : launch_mma_group<64, PKV_BF16_STAGES>(p, grid, st);

@@ -188,11 +188,13 @@ __global__ void PKV_Q8_BOUNDS(NWARPS * kWarp) decode_q8_kernel(const DecodeParam
   uint32_t qf[IK ? 1 : KS][NT][2];
   // INT8 on the integer tensor core (IK): q of head h as the integer
   // Q = rint(q * 2^E_h), E_h chosen so that max_d |q[h][d]| * 2^E_h lies in
-  // [2^22, 2^23), split into three signed bytes Q = p2 * 2^16 + p1 * 2^8 + p0.
-  // Each score is sum_d code * q = 2^-E (2^16 D2 + 2^8 D1 + D0) with Dk the
-  // exact int32 dot products of the codes with the pieces.  Q is exact for
-  // every element within 15 binades of its head's largest (bf16 carries 8
-  // significant bits); smaller elements are rounded at 2^-22 of that largest.
+  // [2^21, 2^22), split into three signed bytes Q = p2 * 2^16 + p1 * 2^8 + p0
+  // (|Q| < 2^22 keeps |p2| <= 65; at 2^23 a largest element with a full bf16
+  // mantissa would need p2 = 128).  Each score is
+  // sum_d code * q = 2^-E (2^16 D2 + 2^8 D1 + D0) with Dk the exact int32 dot
+  // products of the codes with the pieces.  Q is exact for every element
+  // within 14 binades of its head's largest (bf16 carries 8 significant
+  // bits); smaller elements are rounded at 2^-21 of that largest.
   uint32_t qp[IK ? KA : 1][3][NT][2];
   float qc[IK ? NT : 1][2][3];  // per head column: 2^16 2^-E, 2^8 2^-E, 2^-E
   if constexpr (IK) {
@@ -220,10 +222,10 @@ __global__ void PKV_Q8_BOUNDS(NWARPS * kWarp) decode_q8_kernel(const DecodeParam
       }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      // E = 22 - floor(log2 amax), kept within [0, 120] so that 2^E and 2^-E
-      // stay normal fp32 (a head whose largest |q| is below 2^-98 scores ~0)
+      // E = 21 - floor(log2 amax), kept within [0, 120] so that 2^E and 2^-E
+      // stay normal fp32 (a head whose largest |q| is below 2^-99 scores ~0)
       int e_max = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-      int E = amax > 0.f ? 22 - e_max : 0;
+      int E = amax > 0.f ? 21 - e_max : 0;
       E = E < 0 ? 0 : (E > 120 ? 120 : E);
       const float up = __uint_as_float((uint32_t)(E + 127) << 23);  // 2^E
 #pragma unroll
