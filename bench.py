@@ -532,10 +532,17 @@ def kernel_breakdown(call, flush, dev, reps=20):
         _, n = ok(cu.cuGraphGetNodes(graph, 0), "node count")
         nodes, _ = ok(cu.cuGraphGetNodes(graph, n), "nodes")
         deps, byid = {}, {}
+        v2 = getattr(cu, "cuGraphNodeGetDependencies_v2", None)
         for nd in nodes:
             byid[int(nd)] = nd
-            _, nd_n = ok(cu.cuGraphNodeGetDependencies(nd, 0), "deps count")
-            d = ok(cu.cuGraphNodeGetDependencies(nd, nd_n), "deps")[0] if nd_n else []
+            if v2 is not None:
+                # with edge data (programmatic launch edges carry some); an
+                # upper bound on the count, unused entries come back null
+                res = ok(v2(nd, len(nodes)), "deps")
+                d = [x for x in res[0] if x is not None and int(x) != 0]
+            else:
+                _, nd_n = ok(cu.cuGraphNodeGetDependencies(nd, 0), "deps count")
+                d = ok(cu.cuGraphNodeGetDependencies(nd, nd_n), "deps")[0] if nd_n else []
             deps[int(nd)] = [int(x) for x in d]
         order, seen = [], set()
         while len(order) < len(nodes):  # the capture of one stream: a chain

@@ -49,7 +49,10 @@ namespace pkv {
 namespace {
 
 #ifndef PKV_Q8_STAGES
-#define PKV_Q8_STAGES 3
+#define PKV_Q8_STAGES 2
+#endif
+#ifndef PKV_Q8_WARPS
+#define PKV_Q8_WARPS 4
 #endif
 #ifndef PKV_Q8_IMMA
 #define PKV_Q8_IMMA 1
@@ -60,7 +63,7 @@ namespace {
 #ifndef PKV_Q8_HOLD3
 #define PKV_Q8_HOLD3 1
 #endif
-constexpr int kQ8Warps = 4;
+constexpr int kQ8Warps = PKV_Q8_WARPS;
 constexpr int kQ8Stages = PKV_Q8_STAGES;
 
 template <int HD, int NT, int NWARPS, int NSTAGES>
