@@ -39,7 +39,9 @@
 //    value is an fp16 value); no constant to remove.
 // P goes to the tensor core as one fp16 value (11 significant bits; its
 // rounding error, below 2^-11 of each term, is under the bf16 rounding of the
-// output).  The online softmax runs in fp32 with ex2.approx.
+// output).  The online softmax runs in fp32 with ex2.approx; its reference
+// maximum moves only when a score exceeds it by more than 2^8, so most tiles
+// need no warp-wide maximum and no rescale.
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_common.cuh"
@@ -64,6 +66,13 @@ namespace {
 #define PKV_Q8_HOLD3 1
 #endif
 constexpr int kQ8Warps = PKV_Q8_WARPS;
+// The softmax reference maximum moves only when a score exceeds it by more
+// than this (log2 units): P stays below 2^8, far inside fp16, and most tiles
+// skip the warp-wide max reduction and the rescale.
+#ifndef PKV_Q8_LAZY_LOG2
+#define PKV_Q8_LAZY_LOG2 8.0f
+#endif
+constexpr float kLazyLog2 = PKV_Q8_LAZY_LOG2;
 constexpr int kQ8Stages = PKV_Q8_STAGES;
 
 template <int HD, int NT, int NWARPS, int NSTAGES>
@@ -473,20 +482,23 @@ __global__ void PKV_Q8_BOUNDS(NWARPS * kWarp) decode_q8_kernel(const DecodeParam
     }
     }
 
-    // ---- online softmax (tokens g, g+8; heads 2t4, 2t4+1) and P in the B layout
+    // ---- online softmax (tokens g, g+8; heads 2t4, 2t4+1) and P in the B layout.
+    // The reference maximum m_run moves lazily: only when some score of the
+    // tile exceeds it by more than kLazyLog2 (a warp vote; the first tile
+    // always does) is the tile maximum reduced across the warp and the state
+    // rescaled.  Otherwise P = 2^(s - m_run) <= 2^kLazyLog2, and O and l keep
+    // one common reference, so the result is the same softmax.
     uint32_t bh[NT][2];
-    float alpha[NT][2];
-    bool rescale = false;
     const bool va = (mask >> g) & 1u, vb = (mask >> (g + 8)) & 1u;
     const bool all = mask == 0xFFFFu;
+    float sc[NT][4];
+    bool need = false;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float pr[4];
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         if (MHA && jj == 1) {  // one q head per kv head: column 2*t4 + 1 holds none
-          pr[1] = pr[3] = 0.f;
-          alpha[nt][1] = 1.f;
+          sc[nt][1] = sc[nt][3] = -CUDART_INF_F;
           continue;
         }
         float sa = (acc[nt][jj] + acc2[nt][jj]) * rka;
@@ -495,26 +507,30 @@ __global__ void PKV_Q8_BOUNDS(NWARPS * kWarp) decode_q8_kernel(const DecodeParam
           sa = va ? sa : -CUDART_INF_F;
           sb = vb ? sb : -CUDART_INF_F;
         }
-        float mx = fmaxf(sa, sb);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[nt][jj], mx);
-        const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
-        const float a = fast_exp2(m_run[nt][jj] - m_use);
-        pr[jj] = fast_exp2(sa - m_use);
-        pr[jj + 2] = fast_exp2(sb - m_use);
-        l_run[nt][jj] = l_run[nt][jj] * a + (pr[jj] + pr[jj + 2]);
-        m_run[nt][jj] = m_new;
-        alpha[nt][jj] = a;
-        rescale |= (a != 1.f);
+        sc[nt][jj] = sa;
+        sc[nt][jj + 2] = sb;
+        need |= fmaxf(sa, sb) > m_run[nt][jj] + kLazyLog2;
       }
-      // V scales fold into P (a masked token's P is 0: keep its factor finite)
-      const float fva = (all || va) ? rva : 0.f, fvb = (all || vb) ? rvb : 0.f;
-      bh[nt][0] = movmatrix_trans(pack_f16(pr[0] * fva, pr[1] * fva));
-      bh[nt][1] = movmatrix_trans(pack_f16(pr[2] * fvb, pr[3] * fvb));
-    }
-    if (__any_sync(0xffffffffu, rescale)) {
+    if (__any_sync(0xffffffffu, need)) {
+      float alpha[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          if (MHA && jj == 1) {
+            alpha[nt][1] = 1.f;
+            continue;
+          }
+          float mx = fmaxf(sc[nt][jj], sc[nt][jj + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m_run[nt][jj], mx);
+          const float m_use = (m_new == -CUDART_INF_F) ? 0.f : m_new;
+          alpha[nt][jj] = fast_exp2(m_run[nt][jj] - m_use);  // 0 while m_run = -inf
+          l_run[nt][jj] *= alpha[nt][jj];
+          m_run[nt][jj] = m_new;
+        }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -531,6 +547,25 @@ __global__ void PKV_Q8_BOUNDS(NWARPS * kWarp) decode_q8_kernel(const DecodeParam
           o1[nt][3] *= alpha[nt][1];
         }
       }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float pr[4];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        if (MHA && jj == 1) {
+          pr[1] = pr[3] = 0.f;
+          continue;
+        }
+        const float m_use = (m_run[nt][jj] == -CUDART_INF_F) ? 0.f : m_run[nt][jj];
+        pr[jj] = fast_exp2(sc[nt][jj] - m_use);
+        pr[jj + 2] = fast_exp2(sc[nt][jj + 2] - m_use);
+        l_run[nt][jj] += pr[jj] + pr[jj + 2];
+      }
+      // V scales fold into P (a masked token's P is 0: keep its factor finite)
+      const float fva = (all || va) ? rva : 0.f, fvb = (all || vb) ? rvb : 0.f;
+      bh[nt][0] = movmatrix_trans(pack_f16(pr[0] * fva, pr[1] * fva));
+      bh[nt][1] = movmatrix_trans(pack_f16(pr[2] * fvb, pr[3] * fvb));
     }
 
     // ---- O^T[d][head] += V^T * P^T
