@@ -12,6 +12,11 @@ namespace {
 #ifndef PKV_CASCADE_SUFFIX_FIRST
 #define PKV_CASCADE_SUFFIX_FIRST 1
 #endif
+// Prefix slices are planned for about this many CTAs of the shared-prefix
+// pass per SM (over KV heads and row groups).
+#ifndef PKV_PREFIX_CTAS_PER_SM
+#define PKV_PREFIX_CTAS_PER_SM 2
+#endif
 
 constexpr int kMaxChunk = 8192;   // tokens per split (bounds the block-table slice in smem)
 constexpr int kMinChunk = 256;    // below this a split costs more than it balances
@@ -116,8 +121,9 @@ size_t ws_bytes(int num_seqs, int num_q_heads, int head_dim, int splits) {
 
 int map_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
-// Shared-prefix plan: prefix slices (about two CTAs per SM over KV heads and
-// row groups), then the suffix splits of the remaining context.
+// Shared-prefix plan: prefix slices (about PKV_PREFIX_CTAS_PER_SM CTAs per SM
+// over KV heads and row groups), then the suffix splits of the remaining
+// context.
 struct PrefixPlan {
   int ps, pchunk;      // prefix slices and their length
   int splits, chunk;   // suffix splits
@@ -129,7 +135,7 @@ PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head
                        int max_ctx, int prefix_len, pkv_dtype cache_dt, int num_splits) {
   PrefixPlan pl;
   const long long rg = pkv::prefix_row_groups(num_seqs, num_q_heads / num_kv_heads);
-  const long long target = 2LL * sm_count();
+  const long long target = (long long)PKV_PREFIX_CTAS_PER_SM * sm_count();
   long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
   const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;
   const int min_ps = (prefix_len + pkv::kMaxPrefixChunk - 1) / pkv::kMaxPrefixChunk;
