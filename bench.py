@@ -178,7 +178,7 @@ class ClockSampler:
         self._stop.set()
         if self._thread:
             self._thread.join()
-        if self.ok and not self.samples:  # a region shorter than one period
+        if self.ok:  # closing sample: a short region still gets two
             self.sample_once()
 
     def summary(self):
@@ -629,9 +629,11 @@ class StepRunner:
         if args.cascade and self.prefix_len == 0:
             raise SystemExit("--cascade needs a workload with a shared prefix")
         if self.prefix_len:
-            suffix_max = max(self.max_ctx - self.prefix_len, 0)
-            self.splits = args.num_splits or pkv.decode_num_splits(
-                wl.num_seqs, wl.num_kv_heads, wl.head_dim, suffix_max, self.tdt)
+            # the call's own plan (0 = automatic): the prefix pass fills the
+            # suffix decode's last wave, so it splits less than a plain decode
+            self.prefix_slices, self.splits = pkv.shared_prefix_plan(
+                wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, self.max_ctx,
+                self.prefix_len, self.tdt, args.num_splits)
             ws_bytes = pkv.shared_prefix_workspace_size(
                 wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, self.max_ctx,
                 self.prefix_len, self.tdt, self.splits)
@@ -822,7 +824,9 @@ def e2e_overlapped(runner, K, W, world, dev):
             "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / K, 5),
             "overlap": "inputs of step i+1 copied in, and outputs of step i-1 read back, on a "
-                       "second stream while step i runs (double-buffered)"}
+                       "second stream while step i runs (double-buffered)",
+            "l2": "steps back to back as a caller runs them: no L2 flush between steps, and "
+                  "no per-step events"}
 
 
 def measure(name, args, dev, K, W, world, rank, local, peaks, flush, want_e2e=True):
@@ -837,7 +841,12 @@ def measure(name, args, dev, K, W, world, rank, local, peaks, flush, want_e2e=Tr
     kv = wl.kv_bytes()
     value = pdist.whole_job_rate(kv, K, world, sum_ms)
     mean_ms, med_ms = statistics.mean(call_ms), statistics.median(call_ms)
-    achieved = kv / (mean_ms / 1e3) / 1e9
+    # the roofline counts each distinct K/V byte once: with blocks shared
+    # between sequences, the logical bytes (value) include re-reads that HBM
+    # does not serve
+    unique = unique_kv_bytes(wl)
+    roof_bytes = unique if unique < kv else kv
+    achieved = roof_bytes / (mean_ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
     rec = traffic_record(wl)
     roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -846,7 +855,10 @@ def measure(name, args, dev, K, W, world, rank, local, peaks, flush, want_e2e=Tr
             "peak_source": f"{peaks['source']} (hbm_gbs)",
             "decode_ms_mean": round(mean_ms, 5), "decode_ms_median": round(med_ms, 5),
             "decode_ms_min": round(min(call_ms), 5),
-            "frac_median": round(kv / (med_ms / 1e3) / 1e9 / peak, 4)}
+            "frac_median": round(roof_bytes / (med_ms / 1e3) / 1e9 / peak, 4)}
+    if roof_bytes != kv:
+        roof["bytes"] = (f"distinct K/V bytes, {roof_bytes} per call (shared blocks once); the "
+                         f"logical {kv} give {kv / (mean_ms / 1e3) / 1e9:.1f} GB/s (value)")
     if peaks.get("read_gbs"):
         roof["frac_of_same_run_read"] = round(achieved / peaks["read_gbs"], 4)
     if peaks.get("copy_gbs"):
@@ -867,6 +879,7 @@ def measure(name, args, dev, K, W, world, rank, local, peaks, flush, want_e2e=Tr
                                                                        wl.cache_dtype),
         "config": config_dict(wl, args, flushed=flush.enabled),
         "num_splits": runner.splits,
+        **({"prefix_slices": runner.prefix_slices} if runner.prefix_len else {}),
         "pct_of_hbm_peak": round(100 * achieved / peak, 1),
         "tokens_per_s_per_layer": round(wl.num_seqs * world / (ms_per_step / 1e3), 1),
         "model_tokens_per_s": round(wl.num_seqs * world / (ms_per_step / 1e3) / layers, 1),
@@ -910,7 +923,13 @@ def cascade_rooflines(runner, call_ms, peaks, flush, dev):
     runner.check_flags()
     out["kernels"] = kb
     if isinstance(kb, list) and len(kb) == 3:
-        t_pre, t_suf, t_merge = (k["ms_mean"] for k in kb)
+        def ms_of(tag):
+            return next((k["ms_mean"] for k in kb if tag in k["kernel"]), None)
+        t_pre, t_merge = ms_of("prefix_kernel"), ms_of("merge_kernel")
+        t_suf = next((k["ms_mean"] for k in kb
+                      if "prefix_kernel" not in k["kernel"] and "merge_kernel" not in k["kernel"]),
+                     None)
+    if isinstance(kb, list) and len(kb) == 3 and None not in (t_pre, t_suf, t_merge):
         out["prefix_pass"] = {"bound": "tensor", "achieved": round(prefix_flops / (t_pre / 1e3)
                                                                    / 1e12, 1),
                               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",

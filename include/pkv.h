@@ -24,7 +24,7 @@
  *                    pkv_workspace_size, pkv_paged_attention_decode_noalloc
  *   one-launch step  pkv_paged_attention_decode_append (append inside decode)
  *   shared prefix    pkv_paged_attention_decode_shared_prefix[_append],
- *                    pkv_shared_prefix_workspace_size
+ *                    pkv_shared_prefix_workspace_size, pkv_shared_prefix_plan
  *   block manager    pkv_bm_* (host bookkeeping: blocks, ref counts, fork,
  *                    copy-on-write, swap), pkv_copy_blocks (block copies)
  *   misc             pkv_copy, pkv_read, pkv_strerror, pkv_version
@@ -232,6 +232,22 @@ int pkv_paged_attention_decode_append(void* out, const void* q, const void* k, c
 size_t pkv_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                                         int head_dim, int max_context_len, int prefix_len,
                                         pkv_dtype cache_dt, int num_splits);
+
+/*
+ * pkv_shared_prefix_plan - how a shared-prefix call with these sizes divides
+ * its work (host only, launches nothing).  *prefix_slices receives the number
+ * of slices of the shared tokens (one prefix-pass partial each), and
+ * *suffix_splits the number of splits of each sequence's remaining tokens:
+ * num_splits itself, or the automatic choice when num_splits == 0.  That
+ * choice differs from pkv_decode_num_splits of the suffix length: the prefix
+ * pass runs beside the suffix decode and fills its last wave, so the suffix is
+ * not split to fill it.  Either output may be NULL.  Returns PKV_OK, or
+ * PKV_ERR_ARG (a size out of range, prefix_len <= 0, num_q_heads not a
+ * multiple of num_kv_heads).
+ */
+int pkv_shared_prefix_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                           int max_context_len, int prefix_len, pkv_dtype cache_dt,
+                           int num_splits, int* prefix_slices, int* suffix_splits);
 int pkv_paged_attention_decode_shared_prefix(
     void* out, const void* q, pkv_dtype q_dt, const void* k_cache, const void* v_cache,
     pkv_dtype cache_dt, const float* k_scale, const float* v_scale, const int32_t* block_tables,

@@ -9,13 +9,14 @@ from .api import (copy, read, decode_num_splits, kv_cache_append, paged_attentio
                   paged_attention_decode_append, paged_attention_decode_noalloc,
                   paged_attention_decode_shared_prefix,
                   paged_attention_decode_shared_prefix_append,
-                  shared_prefix_workspace_size, workspace_size)
+                  shared_prefix_plan, shared_prefix_workspace_size, workspace_size)
 from .block_manager import BlockManager, copy_blocks
 
 __all__ = ["PkvError", "kv_cache_append", "paged_attention_decode",
            "paged_attention_decode_append",
            "paged_attention_decode_noalloc", "paged_attention_decode_shared_prefix",
            "paged_attention_decode_shared_prefix_append",
-           "shared_prefix_workspace_size", "workspace_size",
-           "decode_num_splits", "copy", "read", "BlockManager", "copy_blocks", "PKV_FLAG_BAD_BLOCK", "PKV_FLAG_BAD_SLOT",
+           "shared_prefix_plan", "shared_prefix_workspace_size", "workspace_size",
+           "decode_num_splits", "copy", "read", "BlockManager", "copy_blocks",
+           "PKV_FLAG_BAD_BLOCK", "PKV_FLAG_BAD_SLOT",
            "PKV_FLAG_CTX_RANGE", "PKV_FLAG_NEG_CTX", "PKV_FLAG_TIMEOUT"]

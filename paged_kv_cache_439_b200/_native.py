@@ -43,6 +43,8 @@ SIGNATURES = {
                                                 _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                                                 _vp]),
     "pkv_shared_prefix_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "pkv_shared_prefix_plan": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_i),
+                                    ctypes.POINTER(_i)]),
     "pkv_paged_attention_decode_shared_prefix": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp,
                                                       _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                                                       _i, _vp, _sz, _i, _vp, _vp]),

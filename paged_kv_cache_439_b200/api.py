@@ -5,8 +5,9 @@ supplies device memory and the current stream.  Names follow include/pkv.h.
 """
 from __future__ import annotations
 
+import ctypes
 import math
-from typing import Optional
+from typing import Optional, Tuple
 
 import torch
 
@@ -293,6 +294,19 @@ def shared_prefix_workspace_size(num_seqs: int, num_q_heads: int, num_kv_heads: 
     return int(N.lib().pkv_shared_prefix_workspace_size(
         num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_len,
         _dtype_code(cache_dtype), num_splits))
+
+
+def shared_prefix_plan(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                       max_context_len: int, prefix_len: int, cache_dtype: torch.dtype,
+                       num_splits: int = 0) -> Tuple[int, int]:
+    """(prefix slices, suffix splits) of a shared-prefix call with these sizes."""
+    ps, ss = ctypes.c_int(0), ctypes.c_int(0)
+    N.check(N.lib().pkv_shared_prefix_plan(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                           max_context_len, prefix_len,
+                                           _dtype_code(cache_dtype), num_splits,
+                                           ctypes.byref(ps), ctypes.byref(ss)),
+            "pkv_shared_prefix_plan")
+    return ps.value, ss.value
 
 
 def paged_attention_decode_shared_prefix(q: torch.Tensor, k_cache: torch.Tensor,

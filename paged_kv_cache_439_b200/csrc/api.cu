@@ -59,14 +59,21 @@ int min_splits(int max_ctx) { return max_ctx <= 0 ? 1 : (max_ctx + kMaxChunk - 1
 //    CTAs fill their last wave at least 90% (equal-length contexts), else the
 //    best-filled one: 128 units on 444 slots take S = 10 (2.9 waves) rather
 //    than 14 (4.04 waves, the fifth nearly empty).
-int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_dtype cache_dt) {
+//  * beside_prefix (the suffix of a shared-prefix call): the prefix pass is
+//    launched behind the suffix decode and its CTAs take the slots that the
+//    decode's last wave leaves free, so with U >= R / 2 the suffix keeps S at
+//    its minimum instead of splitting to fill that wave.
+int auto_splits(int num_seqs, int num_kv_heads, int head_dim, int max_ctx, pkv_dtype cache_dt,
+                bool beside_prefix = false) {
   if (max_ctx <= 0 || num_seqs <= 0) return 1;
   const long long units = (long long)num_seqs * num_kv_heads;
   const long long slots = (long long)sm_count() * pkv::decode_ctas_per_sm_hint(cache_dt, head_dim);
   const int lo = min_splits(max_ctx);
   const int hi = (max_ctx + kMinChunk - 1) / kMinChunk;
   long long want;
-  if (2 * units >= slots) {
+  if (2 * units >= slots && beside_prefix) {
+    want = lo;
+  } else if (2 * units >= slots) {
     want = 1;
     for (int s = 1; s <= 8; ++s) {
       const long long ctas = units * s;
@@ -146,7 +153,7 @@ PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head
   pl.ps = (prefix_len + pl.pchunk - 1) / pl.pchunk;
   const int suffix = max_ctx > prefix_len ? max_ctx - prefix_len : 0;
   int req = num_splits;
-  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, suffix, cache_dt);
+  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, suffix, cache_dt, true);
   plan(suffix, req, &pl.splits, &pl.chunk);
   pl.slots = pl.ps + pl.splits;
   const size_t r = (size_t)num_seqs * num_q_heads * pl.slots;
@@ -382,6 +389,19 @@ size_t pkv_shared_prefix_workspace_size(int num_seqs, int num_q_heads, int num_k
   return plan_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, prefix_len,
                      cache_dt, num_splits)
       .ws;
+}
+
+int pkv_shared_prefix_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                           int max_context_len, int prefix_len, pkv_dtype cache_dt,
+                           int num_splits, int* prefix_slices, int* suffix_splits) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0 ||
+      num_splits < 0 || prefix_len <= 0 || num_q_heads % num_kv_heads != 0)
+    return PKV_ERR_ARG;
+  const PrefixPlan pl = plan_prefix(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                    max_context_len, prefix_len, cache_dt, num_splits);
+  if (prefix_slices) *prefix_slices = pl.ps;
+  if (suffix_splits) *suffix_splits = pl.splits;
+  return PKV_OK;
 }
 
 }  // extern "C"

@@ -249,3 +249,31 @@ def test_split_plans_cover_the_context_in_bounded_chunks(lib, cache_dt):
                 rows = num_seqs * nkv * s
                 want = 0 if s == 1 else ceil(rows * 128 * 4, 256) * 256 + ceil(rows * 4, 256) * 256
                 assert lib.pkv_workspace_size(num_seqs, nkv, nkv, 128, max_ctx, cache_dt, 0) == want
+
+
+def test_shared_prefix_plan(lib):
+    import ctypes
+    ps, ss = ctypes.c_int(0), ctypes.c_int(0)
+
+    def plan(*a):
+        return lib.pkv_shared_prefix_plan(*a, ctypes.byref(ps), ctypes.byref(ss))
+
+    # 64 sequences x 8 KV heads, 4096 shared tokens, suffixes up to 505 tokens:
+    # the (sequence, head) units fill the first wave, and the prefix pass fills
+    # the rest, so the automatic suffix plan does not split
+    assert plan(64, 32, 8, 128, 4601, 4096, 1, 0) == 0
+    assert ss.value == 1 and ps.value >= 1
+    # the plan is the one the workspace size is computed from
+    slots = ps.value + ss.value
+    rows = 64 * 32 * slots
+    assert lib.pkv_shared_prefix_workspace_size(64, 32, 8, 128, 4601, 4096, 1, 0) == \
+        -(-rows * 128 * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
+    # an explicit split count is kept
+    assert plan(64, 32, 8, 128, 4601, 4096, 1, 2) == 0 and ss.value == 2
+    # few units and a long suffix: the suffix is split to occupy the device
+    assert plan(1, 8, 8, 128, 4096 + 20000, 4096, 1, 0) == 0 and ss.value > 1
+    # argument errors; NULL outputs are allowed
+    assert plan(64, 32, 8, 128, 4601, 0, 1, 0) == -1
+    assert plan(64, 30, 8, 128, 4601, 4096, 1, 0) == -1
+    assert plan(0, 32, 8, 128, 4601, 4096, 1, 0) == -1
+    assert lib.pkv_shared_prefix_plan(64, 32, 8, 128, 4601, 4096, 1, 0, None, None) == 0
