@@ -1138,6 +1138,7 @@ def main(argv=None):
             "data": "synthetic (seeded N(0,1) K/V/q shaped like the workload; no weights)",
             "config": head["config"],
             "num_splits": head["num_splits"],
+            **({"prefix_slices": head["prefix_slices"]} if "prefix_slices" in head else {}),
             "pct_of_hbm_peak": head["pct_of_hbm_peak"],
             "tokens_per_s_per_layer": head["tokens_per_s_per_layer"],
             "model_tokens_per_s": head["model_tokens_per_s"],

@@ -9,13 +9,10 @@
 
 namespace {
 
-#ifndef PKV_CASCADE_SUFFIX_FIRST
-#define PKV_CASCADE_SUFFIX_FIRST 1
-#endif
 // Prefix slices are planned for about this many CTAs of the shared-prefix
-// pass per SM (over KV heads and row groups).
-#ifndef PKV_PREFIX_CTAS_PER_SM
-#define PKV_PREFIX_CTAS_PER_SM 2
+// pass per 100 SMs (over KV heads and row groups).
+#ifndef PKV_PREFIX_CTAS_PER_100_SMS
+#define PKV_PREFIX_CTAS_PER_100_SMS 200
 #endif
 
 constexpr int kMaxChunk = 8192;   // tokens per split (bounds the block-table slice in smem)
@@ -128,9 +125,9 @@ size_t ws_bytes(int num_seqs, int num_q_heads, int head_dim, int splits) {
 
 int map_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
-// Shared-prefix plan: prefix slices (about PKV_PREFIX_CTAS_PER_SM CTAs per SM
-// over KV heads and row groups), then the suffix splits of the remaining
-// context.
+// Shared-prefix plan: prefix slices (about PKV_PREFIX_CTAS_PER_100_SMS CTAs
+// per 100 SMs over KV heads and row groups), then the suffix splits of the
+// remaining context.
 struct PrefixPlan {
   int ps, pchunk;      // prefix slices and their length
   int splits, chunk;   // suffix splits
@@ -142,7 +139,7 @@ PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head
                        int max_ctx, int prefix_len, pkv_dtype cache_dt, int num_splits) {
   PrefixPlan pl;
   const long long rg = pkv::prefix_row_groups(num_seqs, num_q_heads / num_kv_heads);
-  const long long target = (long long)PKV_PREFIX_CTAS_PER_SM * sm_count();
+  const long long target = ((long long)PKV_PREFIX_CTAS_PER_100_SMS * sm_count() + 99) / 100;
   long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
   const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;
   const int min_ps = (prefix_len + pkv::kMaxPrefixChunk - 1) / pkv::kMaxPrefixChunk;
@@ -500,16 +497,12 @@ int shared_prefix_impl(
   p.slot_mapping = slot_mapping;
 
   cudaStream_t st = (cudaStream_t)stream;
-#if PKV_CASCADE_SUFFIX_FIRST
   // The suffix decode first; the prefix pass (independent of it: disjoint
   // workspace slots, and the fused append never writes a shared block) is
-  // launched behind it and fills the SMs its last wave leaves idle.
+  // launched behind it and fills the SMs its last wave leaves idle; then the
+  // merge, behind both.
   if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   if (pkv::launch_prefix(p, pp, head_dim, true, st) != cudaSuccess) return PKV_ERR_CUDA;
-#else
-  if (pkv::launch_prefix(p, pp, head_dim, false, st) != cudaSuccess) return PKV_ERR_CUDA;
-  if (pkv::launch_decode(p, cache_dt, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
-#endif
   if (pkv::launch_merge(p, head_dim, st) != cudaSuccess) return PKV_ERR_CUDA;
   return PKV_OK;
 }

@@ -18,10 +18,10 @@
 // slice in 64-token tiles:
 //   S = Q K^T      tcgen05.mma, A = Q and B = K from shared memory (K-major,
 //                  128-byte swizzle), D = S in tensor memory (128 lanes x 64
-//                  fp32 columns);
+//                  fp32 columns, one of two score buffers);
 //   softmax        thread r owns row r: tcgen05.ld of its 64 scores, fp32
-//                  online softmax, P written back to tensor memory as bf16
-//                  hi + lo halves (about 16 significant bits of P);
+//                  online softmax, P written back over S in the same buffer
+//                  as bf16 hi + lo halves (about 16 significant bits of P);
 //   O += P V       tcgen05.mma with A = P from tensor memory and B = V from
 //                  shared memory (head_dim-major), D = O in tensor memory.
 // The running maximum is only moved when a tile's maximum exceeds it by more
@@ -36,13 +36,15 @@
 // MMAs read: Q as a (sequences x heads x 64 columns) box, the K and V tiles
 // as one box per paged block (or 64-token piece of one) and column block, a
 // bad block being read from past the end of the cache (zero fill).  K and V
-// have two-stage rings of their own.  Once every row has read S of tile j
-// into registers, S of tile j + 1 is issued (it runs during tile j's
-// softmax); K tile j + 2 is fetched once S of tile j is done, V tile j + 1
-// once P V of tile j - 1 is done.  Two CTAs share an SM (half of its tensor
-// memory each, at most 168 registers a thread so that both fit), so one CTA's
-// softmax overlaps the other's MMAs.  The softmax keeps eight independent max
-// and sum chains per row.
+// have two-stage rings of their own.  With two score buffers the softmax of
+// tile j never waits for an MMA other than its own S: P_j goes over S_j, S of
+// tile j + 1 is already in the other buffer, and S of tile j + 2 is issued
+// into buffer j % 2 once P V of tile j has read P_j there (it runs during
+// tile j + 1's softmax).  K tile j + 2 is fetched once S of tile j is done, V
+// tile j + 1 once P V of tile j - 1 is done.  Two CTAs share an SM (half of
+// its tensor memory each, at most 168 registers a thread so that both fit),
+// so one CTA's softmax overlaps the other's MMAs.  The softmax keeps eight
+// independent max and sum chains per row.
 #include <math_constants.h>
 
 #include <cuda.h>
@@ -65,6 +67,8 @@ constexpr int kTcTok = kPrefixTokens;  // tokens per tile (MMA N of Q K^T)
 constexpr int kTcStages = 2;
 constexpr float kRescaleLog2 = 8.f;  // move the running max only past 2^8
 constexpr uint64_t kWaitNs = 2000000000ull;  // a wait gives up after 2 s
+constexpr int kTailBarBytes = 128;               // mbarriers, tensor-memory address, failure word
+constexpr int kTailBytes = kTailBarBytes + kTcRows * 8;  // then one workspace row per row
 
 static_assert(kTcTok == 64, "the score row is read as two 32-column loads");
 
@@ -75,14 +79,15 @@ struct TcCfg {
   static constexpr int KV_DB = kTcTok * 128;              // bytes of one K (or V) column block
   static constexpr int Q_BYTES = DB * Q_DB;
   static constexpr int KV_BYTES = DB * KV_DB;            // one K (or V) tile
-  static constexpr int S_COL = 0;                         // tensor-memory columns
-  static constexpr int PH_COL = kTcTok;                   // P hi: 2 bf16 per column
-  static constexpr int PL_COL = kTcTok + kTcTok / 2;      // P lo
+  // tensor-memory columns: two score buffers, S_j in buffer j % 2 (64 fp32
+  // columns) and P_j over it (bf16 hi + lo pairs: 32 columns each), then O
+  static __device__ __forceinline__ uint32_t s_col(int j) { return (uint32_t)((j & 1) * kTcTok); }
   static constexpr int O_COL = 2 * kTcTok;
   static constexpr int COLS_USED = O_COL + HD;
   static constexpr int TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
   // dynamic shared memory: 1 KB alignment slack, Q, the stages, then the
-  // block-table slice, two mbarriers and the tensor-memory address
+  // block-table slice, the mbarriers, the tensor-memory address and failure
+  // word, and the workspace row of each of the 128 rows
   static constexpr int BODY = Q_BYTES + 2 * kTcStages * KV_BYTES;
   static_assert(HD == 64 || HD == 128, "head_dim 64 or 128");
 };
@@ -278,16 +283,22 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
   // Each barrier's waiters must never fall two phases behind it (try_wait.parity
   // would then match the incomplete phase two ahead): every waiter polls a
   // barrier whose next phase cannot complete before that waiter's own next step.
-  const uint32_t bar_sfull = smem_u32(tail);        // S of a tile is in tensor memory (MMA)
-  const uint32_t bar_sfree = smem_u32(tail + 8);    // every row has read S (4 warps; MMA warp)
-  const uint32_t bar_pfull = smem_u32(tail + 16);   // every row has written P (4 warps)
-  const uint32_t bar_odone = smem_u32(tail + 24);   // a tile's P V has been accumulated (MMA)
-  const uint32_t bar_k = smem_u32(tail + 32);       // [2]: K tile (and, first, Q) landed
-  const uint32_t bar_v = smem_u32(tail + 48);       // [2]: V tile landed
-  const uint32_t bar_kfree = smem_u32(tail + 64);   // [2]: S of the stage's K tile is done
-  const uint32_t bar_vfree = smem_u32(tail + 80);   // [2]: P V of the stage's V tile is done
-  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 96);
-  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 100);
+  // Tile j uses score buffer j % 2 and the phase j / 2 of that buffer's pair.
+  const uint32_t bar_sfull = smem_u32(tail);        // [2]: S of a tile is in tensor memory
+  const uint32_t bar_pfull = smem_u32(tail + 16);   // [2]: every row has written P (4 warps)
+  const uint32_t bar_odone = smem_u32(tail + 32);   // a tile's P V has been accumulated (MMA)
+  // Every MMA the CTA issued has completed: one commit after the last issue,
+  // waited once (phase 0), so no later phase can alias it.  The final waits
+  // use it rather than odone, whose last two phases may both have completed
+  // before a waiter polls (the parity of phase n would then match n - 2).
+  const uint32_t bar_done = smem_u32(tail + 40);
+  const uint32_t bar_k = smem_u32(tail + 48);       // [2]: K tile (and, first, Q) landed
+  const uint32_t bar_v = smem_u32(tail + 64);       // [2]: V tile landed
+  const uint32_t bar_kfree = smem_u32(tail + 80);   // [2]: S of the stage's K tile is done
+  const uint32_t bar_vfree = smem_u32(tail + 96);   // [2]: P V of the stage's V tile is done
+  volatile uint32_t* const s_tmem = reinterpret_cast<volatile uint32_t*>(tail + 112);
+  volatile int* const s_fail = reinterpret_cast<volatile int*>(tail + 116);
+  long long* const s_roff = reinterpret_cast<long long*>(tail + kTailBarBytes);  // [kTcRows]
 
   const int kvh = blockIdx.x, split = blockIdx.y, rg = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / kWarp, lane = tid % kWarp;
@@ -300,7 +311,33 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
   const int blk0 = t0 >> p.log2_bs;
   const int ntiles = (t1 - t0 + kTcTok - 1) / kTcTok;
 
-  // ---- set-up: block-table slice, barriers, tensor memory, zeroed Q padding
+  // ---- set-up.  The copy lane initialises the barriers and starts the Q load
+  // at once (it needs no block-table entry); then the block-table slice, the
+  // tensor memory and the zeroed Q padding, all before one CTA barrier.
+  if (copier && lane == 0) {
+    mbar_init(bar_sfull, 1);
+    mbar_init(bar_sfull + 8, 1);
+    mbar_init(bar_pfull, kTcSoftmaxWarps);
+    mbar_init(bar_pfull + 8, kTcSoftmaxWarps);
+    mbar_init(bar_odone, 1);
+    mbar_init(bar_done, 1);
+    mbar_init(bar_kfree, 1);
+    mbar_init(bar_kfree + 8, 1);
+    mbar_init(bar_vfree, 1);
+    mbar_init(bar_vfree + 8, 1);
+    mbar_init(bar_k, 1);
+    mbar_init(bar_k + 8, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_v + 8, 1);
+    *s_fail = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    // Q (rows spc * G of this CTA's sequences) completes on K0's barrier
+    // together with K0; the K0 load adds the arrival
+    mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));
+#pragma unroll
+    for (int db = 0; db < Cfg::DB; ++db)
+      tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
+  }
   {
     const int nphys = ((t1 - 1) >> p.log2_bs) - blk0 + 1;
     for (int i = tid; i < nphys; i += kTcThreads) {
@@ -311,22 +348,6 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       }
       s_phys[i] = b;
     }
-  }
-  if (tid == 0) {
-    mbar_init(bar_sfull, 1);
-    mbar_init(bar_sfree, kTcSoftmaxWarps);
-    mbar_init(bar_kfree, 1);
-    mbar_init(bar_kfree + 8, 1);
-    mbar_init(bar_vfree, 1);
-    mbar_init(bar_vfree + 8, 1);
-    mbar_init(bar_pfull, kTcSoftmaxWarps);
-    mbar_init(bar_odone, 1);
-    mbar_init(bar_k, 1);
-    mbar_init(bar_k + 8, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar_v + 8, 1);
-    *s_fail = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -382,11 +403,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       auto kstage = [&](int j) { return k_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
       auto vstage = [&](int j) { return v_ring + (uint32_t)((j % kTcStages) * Cfg::KV_BYTES); };
       int k_last = -1, v_last = -1;  // last K and V tile issued
-      // Q with K0 first (S of tile 0 waits for them), then V0, K1, V1
-      mbar_add_tx(bar_k, (uint32_t)(Cfg::DB * spc * G * 128));  // Q; K0's load arrives
-#pragma unroll
-      for (int db = 0; db < Cfg::DB; ++db)
-        tma_load_3d(q_sm + (uint32_t)(db * Cfg::Q_DB), &tm_q, db * 64, kvh * G, rg * spc, bar_k);
+      // K0 first (S of tile 0 waits for it and Q), then V0, K1, V1
       load_tile(&tm_k, kstage(0), 0, bar_k);
       load_tile(&tm_v, vstage(0), 0, bar_v);
       k_last = v_last = 0;
@@ -431,64 +448,69 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       const uint64_t dv = smem_desc(v_ring, Cfg::KV_DB, 1024);
       constexpr uint32_t kIdQK = idesc_bf16(kTcRows, kTcTok, 0);
       constexpr uint32_t kIdPV = idesc_bf16(kTcRows, HD, 1);
-      auto issue_qk = [&](int j) {  // S = Q K^T of tile j
+      auto issue_qk = [&](int j) {  // S = Q K^T of tile j into score buffer j % 2
         const uint64_t kb0 = dk + (uint64_t)(((j % kTcStages) * Cfg::KV_BYTES) >> 4);
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {
           const uint32_t koff = (uint32_t)((ks >> 2) * Cfg::KV_DB + (ks & 3) * 32) >> 4;
           const uint32_t qoff = (uint32_t)((ks >> 2) * Cfg::Q_DB + (ks & 3) * 32) >> 4;
-          mma_ss(tmem + Cfg::S_COL, dq + qoff, kb0 + koff, kIdQK, ks > 0);
+          mma_ss(tmem + Cfg::s_col(j), dq + qoff, kb0 + koff, kIdQK, ks > 0);
         }
-        mma_commit(bar_sfull);
+        mma_commit(bar_sfull + 8 * (j % 2));
         mma_commit(bar_kfree + 8 * (j % 2));
       };
-      auto issue_pv = [&](int j) {  // O += P V of tile j
+      auto issue_pv = [&](int j) {  // O += P V of tile j, P (bf16 hi + lo) over S_j
         const uint64_t vb0 = dv + (uint64_t)(((j % kTcStages) * Cfg::KV_BYTES) >> 4);
+        const uint32_t ph = tmem + Cfg::s_col(j), pl = ph + kTcTok / 2;
 #pragma unroll
         for (int kk = 0; kk < kTcTok / 16; ++kk) {
           const uint64_t bd = vb0 + (uint64_t)((kk * 16 * 128) >> 4);
-          mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PH_COL + kk * 8, bd, kIdPV, (j > 0 || kk > 0));
-          mma_ts(tmem + Cfg::O_COL, tmem + Cfg::PL_COL + kk * 8, bd, kIdPV, 1u);
+          mma_ts(tmem + Cfg::O_COL, ph + kk * 8, bd, kIdPV, (j > 0 || kk > 0));
+          mma_ts(tmem + Cfg::O_COL, pl + kk * 8, bd, kIdPV, 1u);
         }
         mma_commit(bar_odone);
         mma_commit(bar_vfree + 8 * (j % 2));
       };
       int n_qk = 0, n_pv = 0;  // tiles whose S = Q K^T / O += P V were issued
-      ok = mbar_wait(bar_k, 0);
-      tc_fence_after();
-      if (ok) {
-        issue_qk(0);
-        n_qk = 1;
-      }
-      for (int j = 0; ok && j < ntiles; ++j) {
-        // every row has read S_j: S of tile j + 1 may overwrite it
-        ok = mbar_wait(bar_sfree, (uint32_t)(j & 1));
-        tc_fence_after();
-        if (ok && j + 1 < ntiles) {
-          ok = mbar_wait(bar_k + 8 * ((j + 1) % 2), (uint32_t)(((j + 1) / 2) & 1));
-          if (ok) {
-            issue_qk(j + 1);
-            n_qk = j + 2;
-          }
-        }
-        // every row has written P_j, V_j has landed: O += P_j V_j
-        if (ok) ok = mbar_wait(bar_pfull, (uint32_t)(j & 1));
-        if (ok) ok = mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
+      // S of tiles 0 and 1 (one per score buffer)
+      for (int j = 0; ok && j < 2 && j < ntiles; ++j) {
+        ok = mbar_wait(bar_k + 8 * j, 0u);
         tc_fence_after();
         if (ok) {
-          issue_pv(j);
-          n_pv = j + 1;
+          issue_qk(j);
+          n_qk = j + 1;
+        }
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        // every row has written P_j, V_j has landed: O += P_j V_j
+        ok = mbar_wait(bar_pfull + 8 * (j % 2), (uint32_t)((j / 2) & 1));
+        if (ok) ok = mbar_wait(bar_v + 8 * (j % 2), (uint32_t)((j / 2) & 1));
+        tc_fence_after();
+        if (!ok) break;
+        issue_pv(j);
+        n_pv = j + 1;
+        // S of tile j + 2 goes into buffer j % 2 once P V of tile j has read
+        // P_j there and K tile j + 2 has landed; it runs during tile j + 1's
+        // softmax
+        if (j + 2 < ntiles) {
+          ok = mbar_wait(bar_odone, (uint32_t)(j & 1));
+          if (ok) ok = mbar_wait(bar_k + 8 * (j % 2), (uint32_t)(((j + 2) / 2) & 1));
+          tc_fence_after();
+          if (ok) {
+            issue_qk(j + 2);
+            n_qk = j + 3;
+          }
         }
       }
       if (!ok) atomicOr(const_cast<int*>(s_fail), kFailWait);
-      // Drain, also after a wait gave up: the last phase committed on each
-      // barrier completes only once every MMA issued before that commit has
-      // finished and its arrive has landed.  Only this lane commits to these
-      // barriers, so none of them can be past the phase waited for.
-      bool drained = true;
-      if (n_qk > 0) drained = drained && mbar_wait(bar_sfull, (uint32_t)((n_qk - 1) & 1));
-      if (n_pv > 0) drained = drained && mbar_wait(bar_odone, (uint32_t)((n_pv - 1) & 1));
-      drained = drained && drain_last(bar_kfree, n_qk - 1) && drain_last(bar_vfree, n_pv - 1);
+      // every MMA issued so far, also after a wait gave up
+      mma_commit(bar_done);
+      // Drain: bar_done completes once every issued MMA has; then the last
+      // phase committed on each ring barrier (its earlier phases were waited
+      // by the softmax or the copy warp, so none of these waits can alias).
+      // Only this lane commits to these barriers.
+      bool drained = mbar_wait(bar_done, 0u) && drain_last(bar_sfull, n_qk - 1) &&
+                     drain_last(bar_kfree, n_qk - 1) && drain_last(bar_vfree, n_pv - 1);
       if (!drained) atomicOr(const_cast<int*>(s_fail), kFailDrain);
     }
   } else {
@@ -498,6 +520,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     const int seq = rg * spc + row / G;
     const bool rvalid = row < spc * G && seq < p.num_seqs;
     const size_t qrow = (size_t)(rvalid ? seq : 0) * p.num_q_heads + kvh * G + row % G;
+    s_roff[row] = rvalid ? (long long)(qrow * p.ws_slots + split) : -1ll;  // workspace row
     int lim = 0;  // tokens of the prefix this row attends to
     if (rvalid) {
       int ctx = p.context_lens[seq];
@@ -509,14 +532,15 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     const float sc = p.scale_log2;
     for (int j = 0; j < ntiles; ++j) {
       const int tt = t0 + j * kTcTok;
-      // ---- scores of tile j, then release S to the next tile's MMA
-      ok = ok && warp_wait(bar_sfull, (uint32_t)(j & 1));
+      const uint32_t sbuf = tmem + lane_base + Cfg::s_col(j);
+      // ---- scores of tile j
+      ok = ok && warp_wait(bar_sfull + 8 * (j % 2), (uint32_t)((j / 2) & 1));
       tc_fence_after();
       float s[kTcTok];
       {
         float a[32], b[32];
-        tmem_ld32(tmem + lane_base + Cfg::S_COL, a);
-        tmem_ld32(tmem + lane_base + Cfg::S_COL + 32, b);
+        tmem_ld32(sbuf, a);
+        tmem_ld32(sbuf + 32, b);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -524,9 +548,6 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
           s[32 + i] = b[i];
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_sfree);
       // valid tokens of this row: inside the slice, below the row's limit, in a good block
       const int nval = max(0, min(t1, lim) - tt);
       bool bad = false;
@@ -549,15 +570,14 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       const float m_new = move ? mt : m_ref;
       const float alpha = move ? fast_exp2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
 
-      // ---- the previous tile's P V must be done: P is overwritten, O may be rescaled
-      if (j > 0) {
-        ok = ok && warp_wait(bar_odone, (uint32_t)((j - 1) & 1));
-        tc_fence_after();
-      }
-      // rare: rescale O in place.  tcgen05.ld/st are warp-collective, so the whole
-      // warp takes this path when any of its rows needs it (alpha = 1 for the rest).
+      // rare: rescale O in place, once the previous tile's P V is done (P_j
+      // goes over S_j in its own buffer, so no other step waits for it).
+      // tcgen05.ld/st are warp-collective, so the whole warp takes this path
+      // when any of its rows needs it (alpha = 1 for the rest).
       const bool need = move && j > 0 && m_ref != -CUDART_INF_F;
       if (__any_sync(0xffffffffu, need)) {
+        ok = ok && warp_wait(bar_odone, (uint32_t)((j - 1) & 1));
+        tc_fence_after();
         const float a_row = need ? alpha : 1.f;
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
@@ -575,7 +595,7 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       m_ref = m_new;
       const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
 
-      // ---- P = 2^(s - m) as bf16 hi + lo, into tensor memory (8 partial sums)
+      // ---- P = 2^(s - m) as bf16 hi + lo over S_j (8 partial sums)
       {
         uint32_t hi[32], lo[32];
         float rs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -589,17 +609,17 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
           lo[i] = pack_bf16(x0 - f.x, x1 - f.y);
         }
         l_run += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-        tmem_st32(tmem + lane_base + Cfg::PH_COL, hi);
-        tmem_st32(tmem + lane_base + Cfg::PL_COL, lo);
+        tmem_st32(sbuf, hi);
+        tmem_st32(sbuf + kTcTok / 2, lo);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull);
+      if (lane == 0) mbar_arrive(bar_pfull + 8 * (j % 2));
       if (!ok) break;
     }
-    // ---- the last P V
-    ok = ok && warp_wait(bar_odone, (uint32_t)((ntiles - 1) & 1));
+    // ---- every MMA, the last P V included, is done
+    ok = ok && warp_wait(bar_done, 0u);
     tc_fence_after();
     if (!ok && lane == 0) atomicOr(const_cast<int*>(s_fail), kFailWait);
     // ---- normalise this slice's partial into shared memory (the K/V rings,
@@ -609,15 +629,18 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
       float4* stage = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES);
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < HD; c += 32) {
-        float o[32];
-        tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o);
+      for (int c = 0; c < HD; c += 64) {
+        float o0[32], o1[32];
+        tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o0);
+        tmem_ld32(tmem + lane_base + Cfg::O_COL + c + 32, o1);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int ch = c / 4 + i;
-          stage[row * CHK + (ch ^ (row & (CHK - 1)))] = make_float4(
-              o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+          const int ch0 = c / 4 + i, ch1 = c / 4 + 8 + i;
+          stage[row * CHK + (ch0 ^ (row & (CHK - 1)))] = make_float4(
+              o0[4 * i] * inv, o0[4 * i + 1] * inv, o0[4 * i + 2] * inv, o0[4 * i + 3] * inv);
+          stage[row * CHK + (ch1 ^ (row & (CHK - 1)))] = make_float4(
+              o1[4 * i] * inv, o1[4 * i + 1] * inv, o1[4 * i + 2] * inv, o1[4 * i + 3] * inv);
         }
       }
       if (rvalid)
@@ -632,12 +655,14 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     // = -inf): the merge then gives it weight 0 and the output stays finite.
     constexpr int CHK = HD / 4;
     constexpr int RPI = 32 / CHK;  // rows per warp store
+    constexpr int ITER = kTcRows / (kTcSoftmaxWarps * RPI);
     const float4* stage = reinterpret_cast<const float4*>(gbase + Cfg::Q_BYTES);
-    for (int rr = warp * RPI + lane / CHK; rr < kTcRows; rr += kTcSoftmaxWarps * RPI) {
-      const int sq = rg * spc + rr / G;
-      if (rr >= spc * G || sq >= p.num_seqs) continue;
-      const size_t slot = ((size_t)sq * p.num_q_heads + kvh * G + rr % G) * p.ws_slots + split;
-      const int ch = lane % CHK;
+    const int ch = lane % CHK;
+#pragma unroll 8
+    for (int it = 0; it < ITER; ++it) {
+      const int rr = (it * kTcSoftmaxWarps + warp) * RPI + lane / CHK;
+      const long long slot = s_roff[rr];
+      if (slot < 0) continue;
       reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] =
           failed ? make_float4(0.f, 0.f, 0.f, 0.f) : stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
       if (failed && ch == 0) p.ws_lse[slot] = -CUDART_INF_F;
@@ -694,7 +719,7 @@ cudaError_t bf16_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
 
 template <int HD>
 int smem_bytes(const PrefixParams& pp) {
-  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + 128;
+  return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + kTailBytes;
 }
 
 // Once per device: the kernel's dynamic shared-memory limit.

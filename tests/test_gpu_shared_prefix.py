@@ -121,6 +121,32 @@ def test_running_max_moves_inside_the_prefix():
     assert g.flags() == 0
 
 
+@pytest.mark.parametrize("bs,moving", [(16, False), (256, False), (16, True)])
+def test_prefix_slices_of_several_tiles(bs, moving):
+    """64 KV heads of group 1 leave few prefix slices, each of several 64-token
+    tiles: both score buffers take turns, S of tile j + 2 is computed behind
+    P V of tile j, and (keys scaled up in two later tiles of the first slice)
+    O is rescaled inside a slice."""
+    prefix = 2048
+    lens = [prefix + x for x in (1, 30, 77, 5, 160, 64, 9, 250)]
+    wl = make_custom(f"sp-tiles-{bs}-{int(moving)}", lens, 64, 64, 128, bs, "bf16", seed=39,
+                     shared_prefix=prefix)
+    ps, _ = pkv.shared_prefix_plan(wl.num_seqs, 64, 64, 128, wl.max_context_len, prefix,
+                                   torch.bfloat16, 0)
+    assert 2 * 64 * ps <= prefix   # two tiles per slice at least
+    if moving:
+        prefix_blocks = wl.block_tables[0, :prefix // bs]
+        blk = wl.prefill_slots // bs
+        for which, factor in ((9, 6.0), (21, 12.0)):   # tiles 2 and 5 of the first slice
+            rows = (blk == prefix_blocks[which]).nonzero().flatten()
+            wl.prefill_k[rows] = (wl.prefill_k[rows].float() * factor).to(wl.prefill_k.dtype)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1):
+        assert_close(_cascade(g, wl, prefix, num_splits=splits), ref, tol_for(wl), wl.name)
+    assert g.flags() == 0
+
+
 def test_repeated_calls_never_stall():
     """Many back-to-back calls, all split choices: the pipeline's hand-offs must
     never deadlock (a stalled CTA gives up after 2 s and sets PKV_FLAG_TIMEOUT)."""
