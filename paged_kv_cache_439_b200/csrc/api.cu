@@ -125,9 +125,10 @@ size_t ws_bytes(int num_seqs, int num_q_heads, int head_dim, int splits) {
 
 int map_cuda(cudaError_t e) { return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA; }
 
-// Shared-prefix plan: prefix slices (about PKV_PREFIX_CTAS_PER_100_SMS CTAs
-// per 100 SMs over KV heads and row groups), then the suffix splits of the
-// remaining context.
+// Shared-prefix plan: the suffix splits of the remaining context, then the
+// prefix slices: about PKV_PREFIX_CTAS_PER_100_SMS CTAs per 100 SMs over KV
+// heads and row groups, and no more than leave the slices and splits of a row
+// within the merge kernel's one-round-trip batch.
 struct PrefixPlan {
   int ps, pchunk;      // prefix slices and their length
   int splits, chunk;   // suffix splits
@@ -143,15 +144,18 @@ PrefixPlan plan_prefix(int num_seqs, int num_q_heads, int num_kv_heads, int head
   long long ps = (target + num_kv_heads * rg - 1) / (num_kv_heads * rg);
   const int max_ps = (prefix_len + pkv::kPrefixTokens - 1) / pkv::kPrefixTokens;
   const int min_ps = (prefix_len + pkv::kMaxPrefixChunk - 1) / pkv::kMaxPrefixChunk;
+  const int suffix = max_ctx > prefix_len ? max_ctx - prefix_len : 0;
+  int req = num_splits;
+  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, suffix, cache_dt, true);
+  plan(suffix, req, &pl.splits, &pl.chunk);
+  // with every partial of a row in one batch, the merge reads them in one
+  // memory round trip
+  if (ps > pkv::kMergeBatch - pl.splits) ps = pkv::kMergeBatch - pl.splits;
   if (ps > max_ps) ps = max_ps;
   if (ps < min_ps) ps = min_ps;  // bounds the block-table slice in shared memory
   if (ps < 1) ps = 1;
   pl.pchunk = round_up((int)((prefix_len + ps - 1) / ps), pkv::kPrefixTokens);
   pl.ps = (prefix_len + pl.pchunk - 1) / pl.pchunk;
-  const int suffix = max_ctx > prefix_len ? max_ctx - prefix_len : 0;
-  int req = num_splits;
-  if (req == 0) req = auto_splits(num_seqs, num_kv_heads, head_dim, suffix, cache_dt, true);
-  plan(suffix, req, &pl.splits, &pl.chunk);
   pl.slots = pl.ps + pl.splits;
   const size_t r = (size_t)num_seqs * num_q_heads * pl.slots;
   pl.ws = align256(r * head_dim * sizeof(float)) + align256(r * sizeof(float));

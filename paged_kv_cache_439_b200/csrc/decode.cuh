@@ -51,6 +51,9 @@ struct PrefixParams {
   int phys_bytes;     // shared-memory bytes for one slice's block-table entries
 };
 constexpr int kPrefixTokens = 64;  // tokens per shared-memory stage
+// Partial rows the merge kernel loads per lane before it knows their weights
+// (one memory round trip for up to this many partials per row).
+constexpr int kMergeBatch = 16;
 constexpr int kMaxPrefixChunk = 8192;  // prefix tokens per slice at most
 
 cudaError_t launch_decode(const DecodeParams& p, pkv_dtype cache_dt, int head_dim,

@@ -21,7 +21,6 @@ namespace {
 // the weights are held one per lane and broadcast with shuffles, 32 slots per
 // round.
 constexpr int kMergeWarps = 4;
-constexpr int kMergeBatch = 16;  // partial rows in flight per lane
 
 template <int HD>
 __global__ void __launch_bounds__(kMergeWarps* kWarp) merge_kernel(const DecodeParams p) {

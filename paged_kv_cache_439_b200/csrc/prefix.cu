@@ -67,6 +67,7 @@ constexpr int kTcTok = kPrefixTokens;  // tokens per tile (MMA N of Q K^T)
 constexpr int kTcStages = 2;
 constexpr float kRescaleLog2 = 8.f;  // move the running max only past 2^8
 constexpr uint64_t kWaitNs = 2000000000ull;  // a wait gives up after 2 s
+constexpr int kOTile = kTcRows * 128;            // staged partial: 128 rows x 32 fp32 columns
 constexpr int kTailBarBytes = 128;               // mbarriers, tensor-memory address, failure word
 constexpr int kTailBytes = kTailBarBytes + kTcRows * 8;  // then one workspace row per row
 
@@ -234,6 +235,21 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// One box of a 4-D tensor map from shared to global memory, in this thread's
+// bulk group.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+// Waits until this thread's bulk stores have completed.
+__device__ __forceinline__ void bulk_store_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Max of 64 values in 8 independent chains.
 __device__ __forceinline__ float max64(const float (&v)[kTcTok]) {
   float m[8];
@@ -268,7 +284,7 @@ template <int HD>
 __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs per SM partition
     prefix_kernel(const DecodeParams p, const PrefixParams pp,
                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o) {
   using Cfg = TcCfg<HD>;
   pdl_trigger();  // the split merge may be scheduled once every CTA has started
   extern __shared__ uint8_t smem_raw[];
@@ -623,10 +639,9 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     tc_fence_after();
     if (!ok && lane == 0) atomicOr(const_cast<int*>(s_fail), kFailWait);
     // ---- normalise this slice's partial into shared memory (the K/V rings,
-    // idle once the last P V is done), so that whole rows go out coalesced
+    // idle once the last P V is done): one 128-byte-swizzled tile of 128 rows
+    // x 32 columns per column block, the layout of the tensor store below
     if (ok) {
-      constexpr int CHK = HD / 4;  // 16-byte chunks per row
-      float4* stage = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES);
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
       for (int c = 0; c < HD; c += 64) {
@@ -634,13 +649,14 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
         tmem_ld32(tmem + lane_base + Cfg::O_COL + c, o0);
         tmem_ld32(tmem + lane_base + Cfg::O_COL + c + 32, o1);
         tmem_wait_ld();
+        float4* t0 = reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES + (c / 32) * kOTile + row * 128);
+        float4* t1 = t0 + kOTile / 16;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int ch0 = c / 4 + i, ch1 = c / 4 + 8 + i;
-          stage[row * CHK + (ch0 ^ (row & (CHK - 1)))] = make_float4(
-              o0[4 * i] * inv, o0[4 * i + 1] * inv, o0[4 * i + 2] * inv, o0[4 * i + 3] * inv);
-          stage[row * CHK + (ch1 ^ (row & (CHK - 1)))] = make_float4(
-              o1[4 * i] * inv, o1[4 * i + 1] * inv, o1[4 * i + 2] * inv, o1[4 * i + 3] * inv);
+          t0[i ^ (row & 7)] = make_float4(o0[4 * i] * inv, o0[4 * i + 1] * inv,
+                                          o0[4 * i + 2] * inv, o0[4 * i + 3] * inv);
+          t1[i ^ (row & 7)] = make_float4(o1[4 * i] * inv, o1[4 * i + 1] * inv,
+                                          o1[4 * i + 2] * inv, o1[4 * i + 3] * inv);
         }
       }
       if (rvalid)
@@ -648,25 +664,35 @@ __global__ void __maxnreg__(168)  // 2 CTAs x 6 warps per SM: 3 warps x 168 regs
     }
   }
 
+  fence_async_smem();  // the staged partial, to the tensor store
   tc_fence_before();
   const bool failed = __syncthreads_or(!ok || *s_fail != 0);
-  if (warp < kTcSoftmaxWarps) {  // coalesced rows of the workspace
+  if (failed) {
     // A slice that gave up writes a defined partial instead (o = 0, log2-sum-exp
     // = -inf): the merge then gives it weight 0 and the output stays finite.
-    constexpr int CHK = HD / 4;
-    constexpr int RPI = 32 / CHK;  // rows per warp store
-    constexpr int ITER = kTcRows / (kTcSoftmaxWarps * RPI);
-    const float4* stage = reinterpret_cast<const float4*>(gbase + Cfg::Q_BYTES);
-    const int ch = lane % CHK;
-#pragma unroll 8
-    for (int it = 0; it < ITER; ++it) {
-      const int rr = (it * kTcSoftmaxWarps + warp) * RPI + lane / CHK;
-      const long long slot = s_roff[rr];
-      if (slot < 0) continue;
-      reinterpret_cast<float4*>(p.ws_o + slot * HD)[ch] =
-          failed ? make_float4(0.f, 0.f, 0.f, 0.f) : stage[rr * CHK + (ch ^ (rr & (CHK - 1)))];
-      if (failed && ch == 0) p.ws_lse[slot] = -CUDART_INF_F;
+    if (warp < kTcSoftmaxWarps) {
+      const int row = tid;
+#pragma unroll 1
+      for (int cb = 0; cb < HD / 32; ++cb)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          reinterpret_cast<float4*>(gbase + Cfg::Q_BYTES + cb * kOTile + row * 128)[i] =
+              make_float4(0.f, 0.f, 0.f, 0.f);
+      const long long slot = s_roff[row];
+      if (slot >= 0) p.ws_lse[slot] = -CUDART_INF_F;
     }
+    fence_async_smem();
+    __syncthreads();
+  }
+  // The partial rows of this slice, (sequence, q head) rows x head_dim, as one
+  // tensor box per 32-column block: workspace dims (head_dim, slot, q head,
+  // sequence); rows of sequences past num_seqs fall outside and are dropped.
+  if (copier && lane == 0) {
+#pragma unroll
+    for (int cb = 0; cb < HD / 32; ++cb)
+      tma_store_4d(&tm_o, smem_u32(gbase + Cfg::Q_BYTES + cb * kOTile), cb * 32, split, kvh * G,
+                   rg * spc);
+    bulk_store_wait();
   }
   if (failed && tid == 0) set_flag(p.err_flag, PKV_FLAG_TIMEOUT);
   // Tensor memory is freed after the bounded drains above, also when one of
@@ -717,6 +743,23 @@ cudaError_t bf16_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The workspace partials as fp32 [num_seqs][num_q_heads][slots][head_dim],
+// stored through 128-byte-swizzled boxes of 32 columns x 1 slot x group heads x
+// sequences-per-CTA.
+cudaError_t ws_map(CUtensorMap* map, float* base, uint64_t hd, uint64_t slots, uint64_t nqh,
+                   uint64_t nseq, uint32_t group, uint32_t spc) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[4] = {hd, slots, nqh, nseq};
+  const cuuint64_t strides[3] = {hd * 4, hd * 4 * slots, hd * 4 * slots * nqh};
+  const cuuint32_t box[4] = {32u, 1u, group, spc};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int HD>
 int smem_bytes(const PrefixParams& pp) {
   return 1024 + TcCfg<HD>::BODY + pp.phys_bytes + kTailBytes;
@@ -750,12 +793,14 @@ cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, bool behind, c
   const int spc = kTcRows / G;
   const int rows_box = p.block_size < kTcTok ? p.block_size : kTcTok;
   const uint64_t cache_rows = (uint64_t)p.num_blocks * p.block_size;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   e = bf16_map(&tq, p.q, HD, p.num_q_heads, p.num_seqs, (uint32_t)G, (uint32_t)spc);
   if (e == cudaSuccess)
     e = bf16_map(&tk, p.k_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
   if (e == cudaSuccess)
     e = bf16_map(&tv, p.v_cache, HD, p.num_kv_heads, cache_rows, 1u, (uint32_t)rows_box);
+  if (e == cudaSuccess)
+    e = ws_map(&to, p.ws_o, HD, p.ws_slots, p.num_q_heads, p.num_seqs, (uint32_t)G, (uint32_t)spc);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.num_kv_heads, pp.prefix_splits, (p.num_seqs + spc - 1) / spc);
@@ -767,7 +812,7 @@ cudaError_t launch(const DecodeParams& p, const PrefixParams& pp, bool behind, c
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = behind ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, prefix_kernel<HD>, p, pp, tq, tk, tv);
+  e = cudaLaunchKernelEx(&cfg, prefix_kernel<HD>, p, pp, tq, tk, tv, to);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -25,7 +25,8 @@ def _cascade(g, wl, prefix_len, context_lens=None, **kw):
 
 
 @pytest.mark.parametrize("group,d,bs", [(4, 128, 16), (1, 128, 16), (8, 128, 16), (16, 64, 16),
-                                        (4, 64, 8), (8, 128, 256), (2, 128, 32)])
+                                        (4, 64, 8), (8, 128, 256), (2, 128, 32), (3, 128, 16),
+                                        (12, 64, 16)])
 def test_shared_prefix_matches_oracle(group, d, bs):
     prefix = 256 if bs == 256 else 4 * bs * 8
     lens = [prefix + x for x in (1, 17, 100, 5, 64, 300)]
