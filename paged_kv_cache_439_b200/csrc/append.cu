@@ -83,6 +83,21 @@ __device__ __forceinline__ uint32_t s8_code(float p) {
   return (uint32_t)q & 0xFFu;
 }
 
+// Four codes of the INT8 rule, packed, for products |p| < 127.5 (every
+// product of a row whose scale 127 / max|x| is finite): adding 1.5 * 2^23 in
+// round-to-nearest-even leaves rint(p) in the low mantissa bits (the sum's
+// unit in the last place is 1), and its low byte is the two's-complement
+// code; no saturation can occur.  An FMA-pipe add and two byte permutes
+// instead of four conversions.
+__device__ __forceinline__ uint32_t s8_codes4(float p0, float p1, float p2, float p3) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint32_t b0 = __float_as_uint(__fadd_rn(p0, kRound));
+  const uint32_t b1 = __float_as_uint(__fadd_rn(p1, kRound));
+  const uint32_t b2 = __float_as_uint(__fadd_rn(p2, kRound));
+  const uint32_t b3 = __float_as_uint(__fadd_rn(p3, kRound));
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
 template <typename T, int EPL>
 __device__ __forceinline__ void widen_vecs(const uint4 (&v)[EPL * sizeof(T) / 16], float (&x)[EPL]) {
   if constexpr (sizeof(T) == 2) {
@@ -162,6 +177,8 @@ __global__ void __launch_bounds__(kQuantThreads)
       for (int o = 1; o < kLanesPerRow; o <<= 1)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const float scale = amax > 0.f ? __fdiv_rn(FP8 ? 448.0f : 127.0f, amax) : 1.0f;
+      // finite max and scale: |x * scale| < 127.5 (the row's common branch)
+      const bool fast = amax <= 3.4e38f && scale <= 3.4e38f;
       uint32_t w[WORDS];
 #pragma unroll
       for (int q = 0; q < WORDS; ++q) {
@@ -170,7 +187,8 @@ __global__ void __launch_bounds__(kQuantThreads)
         if constexpr (FP8)
           w[q] = amax > 0.f ? (f32x2_to_e4m3x2(p0, p1) | (f32x2_to_e4m3x2(p2, p3) << 16)) : 0u;
         else
-          w[q] = s8_code(p0) | (s8_code(p1) << 8) | (s8_code(p2) << 16) | (s8_code(p3) << 24);
+          w[q] = fast ? s8_codes4(p0, p1, p2, p3)
+                      : s8_code(p0) | (s8_code(p1) << 8) | (s8_code(p2) << 16) | (s8_code(p3) << 24);
       }
       if (r < rows) {
         const bool is_v = r >= num_kv_heads;

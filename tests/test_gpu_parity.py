@@ -59,6 +59,29 @@ def test_append_int8_full_13b_bulk(kv):
     assert np.array_equal(bits(g.vs), o.vs.view(np.int32))
 
 
+def test_append_int8_halfway_codes_round_to_even():
+    """A row whose max is 127 has scale exactly 1, so its products are the
+    inputs themselves: halfway values must round to the even code, and the
+    extreme codes must be exact (closed form, no oracle)."""
+    wl = _wl("i8", 4, 2, 128, 16, lens=[8])
+    g = GpuCache(wl)
+    vals = [127.0, 2.5, -3.5, 0.5, -0.5, 126.5, 1.5, -1.5, -127.0, 64.5, -64.5, 0.0]
+    want = [127, 2, -4, 0, 0, 126, 2, -2, -127, 64, -64, 0]
+    k = torch.zeros(1, 2, 128, dtype=torch.bfloat16)
+    k[0, 0, :len(vals)] = torch.tensor(vals, dtype=torch.bfloat16)
+    k[0, 1, :len(vals)] = -torch.tensor(vals, dtype=torch.bfloat16)
+    slot = 5
+    g.append(k, k, torch.tensor([slot], dtype=torch.int64))
+    torch.cuda.synchronize()
+    codes = g.k.cpu().view(torch.int8).numpy().reshape(-1, 2, 128)[slot]
+    assert codes[0, :len(vals)].tolist() == want
+    assert codes[1, :len(vals)].tolist() == [-w if w != 0 else 0 for w in want]
+    assert (codes[:, len(vals):] == 0).all()
+    scales = g.ks.cpu().numpy().reshape(-1, 2, 16)[slot // 16, :, slot % 16]
+    assert scales.tolist() == [1.0, 1.0]
+    assert g.flags() == 0
+
+
 def test_append_skips_negative_and_flags_bad_slots():
     wl = _wl("bf16", 4, 2, 64, 16, lens=[20])
     g = GpuCache(wl)
