@@ -863,6 +863,10 @@ def measure(name, args, dev, K, W, world, rank, local, peaks, flush, want_e2e=Tr
         roof["frac_of_same_run_read"] = round(achieved / peaks["read_gbs"], 4)
     if peaks.get("copy_gbs"):
         roof["frac_of_same_run_copy"] = round(achieved / peaks["copy_gbs"], 4)
+    roof["headline"] = ("frac: achieved over peak (peak_source); the same achieved rate over this "
+                        "run's streaming-read probe (the decode only reads K/V) is "
+                        "frac_of_same_run_read, over its copy probe (read + write bytes) "
+                        "frac_of_same_run_copy")
     if runner.prefix_len:
         roof["kernel"] = ("pkv_paged_attention_decode_shared_prefix" +
                           ("_append" if runner.fused else "") +
