@@ -42,7 +42,8 @@ def _same_cache(a, b):
 
 
 @pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8"])
-@pytest.mark.parametrize("group,d,bs", [(4, 128, 16), (1, 64, 16), (8, 128, 256), (16, 64, 8)])
+@pytest.mark.parametrize("group,d,bs", [(4, 128, 16), (1, 64, 16), (8, 128, 256), (16, 64, 8),
+                                        (3, 128, 16), (12, 64, 16)])
 def test_fused_step_equals_append_then_decode(cache_dtype, group, d, bs):
     lens = [1, 17, 100, 333, 64, 1024]
     wl = make_custom(f"fused-{cache_dtype}-{group}-{d}-{bs}", lens, 2 * group, 2, d, bs,

@@ -126,6 +126,22 @@ def test_decode_dtype_group_headdim(cache_dtype, group, d):
     assert g.flags() == 0
 
 
+@pytest.mark.parametrize("cache_dtype", ["bf16", "i8", "fp8", "f32"])
+@pytest.mark.parametrize("group", [2, 3, 6, 12])
+def test_decode_groups_not_filling_the_head_tile(cache_dtype, group):
+    """Groups that leave head columns of the mma n-tile (8 heads, or 16 with two
+    tiles above 8) unused: those columns are masked and never written."""
+    nkv = 3
+    wl = _wl(cache_dtype, nkv * group, nkv, 128, 16, seed=12,
+             outlier_prob=0.01 if cache_dtype in ("i8", "fp8") else 0)
+    g = GpuCache(wl).fill()
+    ref = OracleCache(wl).fill().decode()
+    for splits in (0, 1, 3):
+        out = g.decode(num_splits=splits)
+        assert_close(out, ref, tol_for(wl), f"{wl.name} splits={splits}")
+    assert g.flags() == 0
+
+
 @pytest.mark.parametrize("cache_dtype,bs", [("bf16", 8), ("bf16", 32), ("bf16", 256),
                                             ("i8", 8), ("i8", 256), ("fp8", 8), ("fp8", 256),
                                             ("f32", 128)])
