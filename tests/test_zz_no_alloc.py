@@ -29,10 +29,12 @@ def _cases():
         make_custom("noalloc-mha-int8", [700, 2049, 33], 4, 4, 128, 16, "i8", seed=22,
                     outlier_prob=0.01),
         make_custom("noalloc-gqa4-bs256", [5000, 260, 999], 8, 2, 64, 256, "bf16", seed=23),
+        make_custom("noalloc-gqa2-fp8", [1800, 2600, 90], 4, 2, 128, 16, "fp8", seed=24,
+                    outlier_prob=0.01),
     ]
 
 
-@pytest.mark.parametrize("idx", [0, 1, 2])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3])
 @pytest.mark.parametrize("splits", [0, 5])
 def test_noalloc_matches_workspace_entry_point(idx, splits):
     import paged_kv_cache_439_b200 as pkv
