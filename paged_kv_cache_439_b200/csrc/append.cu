@@ -180,15 +180,23 @@ __global__ void __launch_bounds__(kQuantThreads)
       // finite max and scale: |x * scale| < 127.5 (the row's common branch)
       const bool fast = amax <= 3.4e38f && scale <= 3.4e38f;
       uint32_t w[WORDS];
+      if (FP8 || fast) {
 #pragma unroll
-      for (int q = 0; q < WORDS; ++q) {
-        const float p0 = __fmul_rn(x[4 * q], scale), p1 = __fmul_rn(x[4 * q + 1], scale);
-        const float p2 = __fmul_rn(x[4 * q + 2], scale), p3 = __fmul_rn(x[4 * q + 3], scale);
-        if constexpr (FP8)
-          w[q] = amax > 0.f ? (f32x2_to_e4m3x2(p0, p1) | (f32x2_to_e4m3x2(p2, p3) << 16)) : 0u;
-        else
-          w[q] = fast ? s8_codes4(p0, p1, p2, p3)
-                      : s8_code(p0) | (s8_code(p1) << 8) | (s8_code(p2) << 16) | (s8_code(p3) << 24);
+        for (int q = 0; q < WORDS; ++q) {
+          const float p0 = __fmul_rn(x[4 * q], scale), p1 = __fmul_rn(x[4 * q + 1], scale);
+          const float p2 = __fmul_rn(x[4 * q + 2], scale), p3 = __fmul_rn(x[4 * q + 3], scale);
+          if constexpr (FP8)
+            w[q] = amax > 0.f ? (f32x2_to_e4m3x2(p0, p1) | (f32x2_to_e4m3x2(p2, p3) << 16)) : 0u;
+          else
+            w[q] = s8_codes4(p0, p1, p2, p3);
+        }
+      } else {  // INT8 row whose scale is not finite (max |x| infinite, NaN or below 2^-126 * 127)
+#pragma unroll
+        for (int q = 0; q < WORDS; ++q) {
+          const float p0 = __fmul_rn(x[4 * q], scale), p1 = __fmul_rn(x[4 * q + 1], scale);
+          const float p2 = __fmul_rn(x[4 * q + 2], scale), p3 = __fmul_rn(x[4 * q + 3], scale);
+          w[q] = s8_code(p0) | (s8_code(p1) << 8) | (s8_code(p2) << 16) | (s8_code(p3) << 24);
+        }
       }
       if (r < rows) {
         const bool is_v = r >= num_kv_heads;
