@@ -100,3 +100,22 @@ def test_reference_config_equals_the_gpu_arm_config_keys():
     assert "num_splits" not in c and c["workload"] == "tiny"
     assert c == bench.config_dict(make_workload("tiny"), args, flushed=True)
     assert bench.parse([]).workload == "llama2-70b-gqa"
+
+
+def test_traffic_record_is_used_only_for_the_sources_it_was_captured_on():
+    """A committed ncu traffic record reaches the bench line only while the
+    decode kernel's sources still hash to the digest stored with it."""
+    from types import SimpleNamespace
+    b = _bench_module()
+    recs = json.load(open(os.path.join(ROOT, "profiles", "decode_traffic.json")))["records"]
+    assert recs
+    for rec in recs:
+        wl = SimpleNamespace(name=rec["workload"], block_size=rec["block_size"],
+                             cache_dtype=rec["cache_dtype"])
+        assert rec["kernel_sources"] == b.kernel_sources(rec["cache_dtype"])
+        b.kernel_source_digest = lambda dt, d=rec["kernel_sources_sha256_16"]: d
+        assert b.traffic_record(wl) == rec
+        b.kernel_source_digest = lambda dt: "0" * 16      # the sources changed
+        assert b.traffic_record(wl) is None
+        # traffic within 1% of the algorithmic bytes: no re-reads
+        assert 0.98 < rec["traffic_over_algorithmic"] < 1.02
